@@ -1,0 +1,190 @@
+"""CPU oracle for the DeepSeek Sparse Attention (DSA) hot path — TEST INFRASTRUCTURE.
+
+Only the tests, the package's smoke check and the benchmark's CPU-baseline leg
+may import this module.  The CUDA library never calls it, and it shares no code
+with the CUDA path: it decodes FP8 and BF16 from their bit definitions, walks
+the block table itself and computes everything in float64 with plain numpy.
+
+What it computes, step by step, follows the DSA description on the pages
+"DeepSeek V3.2-Exp Cuts Prolonged-Context Costs With DeepSeek Sparse Attention
+(DSA) Whereas Sustaining Benchmark Parity" (section "FP8 index -> top-k
+selection -> sparse core attention") and its Spanish translation
+"Deepseek v3.2-Exp reduce los costos de contexto largo ..." (same section):
+
+  (1) lightning indexer: for query token t and every preceding token s (s <= pos(t))
+          I[t,s] = sum_j w[t,j] * ReLU(qhat[t,j,:] . khat[s,:])
+      over a few FP8 indexer heads j (the printed formula is garbled on the pages;
+      this is the reading fixed by the workload definition that accompanies them);
+  (2) fine-grained selection: the top-k (k = 2048) entries of I[t,:];
+  (3) standard softmax attention over only the selected entries, MLA in MQA mode:
+      every query head h attends to the same 576-wide latent rows, whose first 512
+      values are the value vector.
+
+Readings of points the pages leave open (each one is listed in the design doc):
+  * causality includes the token itself: s ranges over [0, pos(t)];
+  * ties in (2) go to the smaller position s; fewer than k valid keys -> all of them;
+  * FP8 is e4m3 "fn" (bias 7, no infinities, S.1111.111 = NaN, max 448), one fp32
+    scale per token; BF16 is the upper half of an IEEE fp32;
+  * the softmax uses max subtraction and returns LSE = max + log(sum exp).
+
+Every function below is pinned by tests/test_oracle_pins.py (closed forms,
+brute force on tiny inputs, library special cases and invariants).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+PAGE = 64
+
+
+# --------------------------------------------------------------------------------------
+# storage formats
+# --------------------------------------------------------------------------------------
+
+def decode_e4m3(b) -> np.ndarray:
+    """FP8 e4m3 ("fn") bytes -> float64 from the bit layout S.EEEE.MMM.
+
+    exponent bias 7; exponent field 0 is subnormal (value = M/8 * 2^-6);
+    S.1111.111 is NaN (the format has no infinities); max finite 448.
+    """
+    b = np.asarray(b, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = b & 0x7
+    normal = (1.0 + m / 8.0) * np.exp2(e - 7.0)
+    sub = (m / 8.0) * np.exp2(-6.0)
+    val = sign * np.where(e == 0, sub, normal)
+    return np.where((e == 0xF) & (m == 0x7), np.nan, val)
+
+
+def decode_bf16(u) -> np.ndarray:
+    """BF16 bit patterns (uint16) -> float64: they are the upper 16 bits of an fp32."""
+    u = np.asarray(u, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------------------
+# paged cache addressing
+# --------------------------------------------------------------------------------------
+
+def logical_rows(block_table, b: int, n: int, page: int = PAGE) -> np.ndarray:
+    """Physical cache rows of logical tokens 0..n-1 of sequence b.
+
+    Token s lives in physical block block_table[b][s // page] at slot s % page
+    (64-token pages, "Quick guide to run it locally": --page-size 64).
+    """
+    s = np.arange(n, dtype=np.int64)
+    return np.asarray(block_table)[b, s // page].astype(np.int64) * page + s % page
+
+
+# --------------------------------------------------------------------------------------
+# (1) lightning indexer
+# --------------------------------------------------------------------------------------
+
+def indexer_logits_row(k8, k_scale, block_table, b: int, pos: int, q8_t, q_scale_t, w_t,
+                       page: int = PAGE) -> np.ndarray:
+    """I[t, s] for s = 0..pos of one query token t of sequence b (float64, length pos+1).
+
+    qhat[j,:] = decode(q8[t,j,:]) * q_scale[t];  khat[s,:] = decode(k8[s,:]) * k_scale[s];
+    I[t,s] = sum_j w[t,j] * max(0, qhat[j,:] . khat[s,:]).
+    """
+    rows = logical_rows(block_table, b, pos + 1, page)
+    khat = decode_e4m3(np.asarray(k8)[rows]) * np.asarray(k_scale, np.float64)[rows, None]
+    qhat = decode_e4m3(q8_t) * float(q_scale_t)  # [H_I, D_I]
+    dots = khat @ qhat.T  # [pos+1, H_I]
+    return np.maximum(dots, 0.0) @ np.asarray(w_t, np.float64)
+
+
+def indexer_logits(cache, qs) -> list:
+    """Indexer rows for every query token of a call: list of float64 arrays."""
+    return [indexer_logits_row(cache.k8, cache.k_scale, cache.block_table,
+                               int(qs.tok_seq[t]), int(qs.tok_pos[t]),
+                               qs.q8[t], qs.q_scale[t], qs.w[t], cache.page)
+            for t in range(qs.n_tokens)]
+
+
+# --------------------------------------------------------------------------------------
+# (2) fine-grained token selection
+# --------------------------------------------------------------------------------------
+
+def topk_select(row, k: int) -> np.ndarray:
+    """Positions of the n = min(k, len(row)) largest entries, ascending by position.
+
+    Ordered by (value descending, position ascending): among equal values the
+    smaller position wins.
+    """
+    row = np.asarray(row, dtype=np.float64)
+    n = min(int(k), row.shape[0])
+    order = np.lexsort((np.arange(row.shape[0]), -row))  # primary: -value; secondary: s
+    return np.sort(order[:n]).astype(np.int64)
+
+
+def kth_value(row, k: int) -> float:
+    """The n-th largest value of the row, n = min(k, len(row))."""
+    row = np.sort(np.asarray(row, np.float64))[::-1]
+    return float(row[min(int(k), row.shape[0]) - 1])
+
+
+# --------------------------------------------------------------------------------------
+# (3) sparse MLA attention in MQA mode
+# --------------------------------------------------------------------------------------
+
+def sparse_mla_attn_token(kv, block_table, b: int, q_t, sel, scale: float, d_v: int,
+                          page: int = PAGE):
+    """Attention of one query token over its selected logical positions ``sel``.
+
+    q_t: BF16 bits [H, D_kv]; kv: BF16 bits [rows, D_kv]; sel: logical positions.
+    z[h,s] = scale * (q[h,:] . kv[s,:])  over the full latent+rope width;
+    p = softmax_s(z) with max subtraction;  O[h,:] = sum_s p[h,s] * kv[s, :d_v];
+    LSE[h] = max_s z + log(sum_s exp(z - max)).
+    Returns (O float64 [H, d_v], LSE float64 [H]).
+    """
+    sel = np.asarray(sel, dtype=np.int64)
+    bt = np.asarray(block_table)
+    rows = bt[b, sel // page].astype(np.int64) * page + sel % page
+    kvh = decode_bf16(np.asarray(kv)[rows])  # [n, D_kv]
+    qh = decode_bf16(q_t)  # [H, D_kv]
+    z = scale * (qh @ kvh.T)  # [H, n]
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    l = e.sum(axis=1, keepdims=True)
+    out = (e / l) @ kvh[:, :d_v]
+    lse = (m + np.log(l))[:, 0]
+    return out, lse
+
+
+def softmax_weights(kv, block_table, b, q_t, sel, scale, page: int = PAGE):
+    """The attention probabilities p[h, i] of ``sparse_mla_attn_token`` (rows sum to 1)."""
+    sel = np.asarray(sel, dtype=np.int64)
+    bt = np.asarray(block_table)
+    rows = bt[b, sel // page].astype(np.int64) * page + sel % page
+    z = scale * (decode_bf16(q_t) @ decode_bf16(np.asarray(kv)[rows]).T)
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    return e / e.sum(axis=1, keepdims=True)
+
+
+# --------------------------------------------------------------------------------------
+# the whole path and its work counters
+# --------------------------------------------------------------------------------------
+
+def dsa_forward_token(cache, qs, t: int, topk: int, scale: float, d_v: int):
+    """(1) -> (2) -> (3) for query token t.  Returns (logits, sel, O, LSE)."""
+    b, pos = int(qs.tok_seq[t]), int(qs.tok_pos[t])
+    logits = indexer_logits_row(cache.k8, cache.k_scale, cache.block_table, b, pos,
+                                qs.q8[t], qs.q_scale[t], qs.w[t], cache.page)
+    sel = topk_select(logits, topk)
+    out, lse = sparse_mla_attn_token(cache.kv, cache.block_table, b, qs.q[t], sel,
+                                     scale, d_v, cache.page)
+    return logits, sel, out, lse
+
+
+def work_counts(tok_pos, topk: int):
+    """(indexer pairs, attention pairs) of one call.
+
+    The indexer scores every preceding token: sum_t (pos(t)+1), quadratic in L for
+    a causal prefill.  Attention visits only the selected ones: sum_t min(k, pos(t)+1),
+    linear in L once L >> k — the O(L^2) -> O(L k) change the pages describe.
+    """
+    p = np.asarray(tok_pos, dtype=np.int64) + 1
+    return int(p.sum()), int(np.minimum(p, int(topk)).sum())

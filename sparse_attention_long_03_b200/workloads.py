@@ -1,0 +1,354 @@
+"""Seeded synthetic inputs for the DeepSeek Sparse Attention (DSA) hot path.
+
+This module is the one thing the CUDA path and the CPU oracle share: it draws
+random numbers and lays them out the way the paged caches are stored.  It holds
+none of the method's arithmetic (no index logits, no selection, no softmax).
+Storage conversions (fp32 -> FP8 e4m3 bytes, fp32 -> BF16 bits) use torch's own
+casts, so that the oracle's bit-level decoders are checked against an
+independent encoder.
+
+Workloads follow the five configurations the DSA pages are measured on
+("DeepSeek V3.2-Exp Cuts Prolonged-Context Costs ...", section
+"FP8 index -> top-k selection -> sparse core attention": FP8 indexer with few
+heads and ReLU, top-k = 2048, MLA in MQA mode; "DeepSeek V3.2-Exp: Sparse
+Attention, Long Context, and Cheaper API", section "Quick guide to run it
+locally": 64-token pages):
+
+  tiny             batch 1, L=512, queries at positions 508..511, indexer 4x32,
+                   k=32, 8 heads, latent 80 (64 + 16 rope), w ~ U(0,1)/4
+  decode_32k       batch 8, one query each at position L-1, L=32768,
+                   indexer 64x128, k=2048, 128 heads, latent 576 (512 + 64)
+  decode_128k      batch 4, L ~ U[65536, 131072], 16 planted keys per query
+  prefill_16k      batch 1, 16384 causal queries, all values ~ N(0,1)
+  chunked_64k      batch 2, L=65536 in 4096-token chunks, index keys copied
+                   from 8 distinct FP8 vectors (heavy logit ties)
+
+Draw order (every stream is numpy ``default_rng`` keyed by a tuple, so any
+piece can be regenerated alone):
+  [seed, 0]            sequence lengths, then the physical block permutation
+  [seed, 1, b, blk]    index keys of sequence b, logical block blk (64 tokens)
+  [seed, 2, b, blk]    latent KV rows of sequence b, logical block blk
+  [seed, 3, b, p//256] indexer query q8 (fp32 draw) and w, 256 positions/draw
+  [seed, 4, b, p//256] attention query q (bf16), 256 positions per draw
+  [seed, 5, b]         planted-key positions (decode_128k); [seed, 5, b, 1] their noise
+  [seed, 6]            the 8 tie vectors (chunked_64k)
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+PAGE = 64
+FP8_MAX = 448.0
+POISON_FP8 = 0x7F  # e4m3 NaN
+POISON_BF16 = 0x7FC0  # bf16 quiet NaN
+POS_BLOCK = 256  # positions per query draw
+
+
+@dataclasses.dataclass(frozen=True)
+class Config:
+    name: str
+    seed: int
+    batch: int
+    n_idx_heads: int  # H_I
+    idx_dim: int  # D_I
+    topk: int
+    n_heads: int  # H
+    d_kv: int  # latent + rope
+    d_v: int  # latent (value) width
+    w_dist: str  # "uniform_quarter" | "normal_eighth" | "normal"
+    lens: Optional[Sequence[int]] = None  # fixed lengths; None -> drawn
+    len_range: Optional[tuple] = None
+    planted: int = 0
+    tie_vectors: int = 0
+    chunk: int = 0  # chunk size for chunked prefill (0 = none)
+    queries: str = "decode"  # "decode" | "tail4" | "prefill"
+
+    @property
+    def scale(self) -> float:
+        # softmax scale: 1/sqrt(80) for the tiny case, 1/sqrt(192) otherwise
+        return 1.0 / math.sqrt(80.0) if self.d_kv == 80 else 1.0 / math.sqrt(192.0)
+
+
+CONFIGS = {
+    "tiny": Config("tiny", 0, 1, 4, 32, 32, 8, 80, 64, "uniform_quarter",
+                   lens=(512,), queries="tail4"),
+    "decode_32k": Config("decode_32k", 1, 8, 64, 128, 2048, 128, 576, 512,
+                         "normal_eighth", lens=(32768,) * 8),
+    "decode_128k": Config("decode_128k", 2, 4, 64, 128, 2048, 128, 576, 512,
+                          "normal_eighth", len_range=(65536, 131072), planted=16),
+    "prefill_16k": Config("prefill_16k", 3, 1, 64, 128, 2048, 128, 576, 512,
+                          "normal", lens=(16384,), queries="prefill"),
+    "chunked_64k": Config("chunked_64k", 4, 2, 64, 128, 2048, 128, 576, 512,
+                          "normal_eighth", lens=(65536, 65536), tie_vectors=8,
+                          chunk=4096, queries="prefill"),
+}
+
+
+@dataclasses.dataclass
+class PagedCache:
+    """Host copies of the paged caches, exactly the bytes the GPU reads.
+
+    k8        uint8  [num_blocks*64, D_I]   FP8 e4m3 index keys
+    k_scale   fp32   [num_blocks*64]        per-token index-key scale
+    kv        uint16 [num_blocks*64, D_kv]  BF16 latent rows (bits)
+    block_table int32 [B, max_blocks]       physical block of (seq, logical block); -1 = unused
+    seq_lens  int32  [B]
+    """
+
+    k8: np.ndarray
+    k_scale: np.ndarray
+    kv: Optional[np.ndarray]
+    block_table: np.ndarray
+    seq_lens: np.ndarray
+    page: int = PAGE
+
+    @property
+    def num_blocks(self) -> int:
+        return self.k8.shape[0] // self.page
+
+    def phys_row(self, b: int, s: np.ndarray) -> np.ndarray:
+        s = np.asarray(s)
+        return self.block_table[b, s // self.page].astype(np.int64) * self.page + s % self.page
+
+
+@dataclasses.dataclass
+class Queries:
+    """Host copies of one call's query tokens.
+
+    tok_seq int32 [T], tok_pos int32 [T]
+    q8      uint8 [T, H_I, D_I]  FP8 e4m3 indexer query
+    q_scale fp32  [T]            per-token scale of q8 (over all H_I*D_I values)
+    w       fp32  [T, H_I]       indexer head weights
+    q       uint16 [T, H, D_kv]  BF16 attention query (bits); None if not drawn
+    """
+
+    tok_seq: np.ndarray
+    tok_pos: np.ndarray
+    q8: np.ndarray
+    q_scale: np.ndarray
+    w: np.ndarray
+    q: Optional[np.ndarray]
+
+    @property
+    def n_tokens(self) -> int:
+        return int(self.tok_seq.shape[0])
+
+
+def _rng(*key: int) -> np.random.Generator:
+    return np.random.default_rng([int(k) for k in key])
+
+
+def to_e4m3_bytes(x: np.ndarray) -> np.ndarray:
+    """fp32 values already inside [-448, 448] -> e4m3fn bytes (torch cast, RNE)."""
+    t = torch.from_numpy(np.ascontiguousarray(np.clip(x, -FP8_MAX, FP8_MAX), dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def quantize_per_row(x: np.ndarray):
+    """Per-row FP8 storage: scale = amax/448 (1 if amax == 0), bytes = e4m3(x/scale).
+
+    x: fp32 [R, n].  Returns (bytes uint8 [R, n], scale fp32 [R]).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.abs(x).max(axis=1)
+    scale = np.where(amax > 0, amax / np.float32(FP8_MAX), np.float32(1.0)).astype(np.float32)
+    return to_e4m3_bytes(x / scale[:, None]), scale
+
+
+def e4m3_values_torch(b: np.ndarray) -> np.ndarray:
+    """Decoded e4m3 bytes via torch (used only to aim the planted keys)."""
+    t = torch.from_numpy(np.ascontiguousarray(b, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float32).numpy()
+
+
+def _layout(cfg: Config):
+    """Sequence lengths, then a random permutation of all physical blocks."""
+    rng = _rng(cfg.seed, 0)
+    if cfg.lens is not None:
+        lens = np.asarray(cfg.lens, dtype=np.int32)
+    else:
+        lo, hi = cfg.len_range
+        lens = rng.integers(lo, hi, size=cfg.batch, endpoint=True).astype(np.int32)
+    nblk = [(int(L) + PAGE - 1) // PAGE for L in lens]
+    perm = rng.permutation(sum(nblk)).astype(np.int32)
+    return lens, nblk, perm
+
+
+def seq_lens_of(cfg: Config) -> np.ndarray:
+    return _layout(cfg)[0]
+
+
+def block_table_of(cfg: Config) -> np.ndarray:
+    _, nblk, perm = _layout(cfg)
+    bt = np.full((cfg.batch, max(nblk)), -1, dtype=np.int32)
+    o = 0
+    for b, n in enumerate(nblk):
+        bt[b, :n] = perm[o:o + n]
+        o += n
+    return bt
+
+
+def _w_draw(cfg: Config, rng: np.random.Generator, n: int) -> np.ndarray:
+    h = cfg.n_idx_heads
+    if cfg.w_dist == "uniform_quarter":
+        return (rng.random((n, h), dtype=np.float32) / 4).astype(np.float32)
+    if cfg.w_dist == "normal_eighth":
+        return (rng.standard_normal((n, h), dtype=np.float32) / 8).astype(np.float32)
+    return rng.standard_normal((n, h), dtype=np.float32)
+
+
+def _idx_query_block(cfg: Config, b: int, blk: int):
+    """q8 / q_scale / w for positions [blk*256, blk*256+256) of sequence b."""
+    rng = _rng(cfg.seed, 3, b, blk)
+    qf = rng.standard_normal((POS_BLOCK, cfg.n_idx_heads * cfg.idx_dim), dtype=np.float32)
+    w = _w_draw(cfg, rng, POS_BLOCK)
+    q8, qs = quantize_per_row(qf)
+    return q8.reshape(POS_BLOCK, cfg.n_idx_heads, cfg.idx_dim), qs, w
+
+
+def _attn_query_block(cfg: Config, b: int, blk: int) -> np.ndarray:
+    rng = _rng(cfg.seed, 4, b, blk)
+    qf = rng.standard_normal((POS_BLOCK, cfg.n_heads, cfg.d_kv), dtype=np.float32)
+    return to_bf16_bits(qf)
+
+
+def make_queries(cfg: Config, tok_seq, tok_pos, with_q: bool = True) -> Queries:
+    tok_seq = np.asarray(tok_seq, dtype=np.int32)
+    tok_pos = np.asarray(tok_pos, dtype=np.int32)
+    T = tok_seq.shape[0]
+    q8 = np.empty((T, cfg.n_idx_heads, cfg.idx_dim), np.uint8)
+    qs = np.empty((T,), np.float32)
+    w = np.empty((T, cfg.n_idx_heads), np.float32)
+    q = np.empty((T, cfg.n_heads, cfg.d_kv), np.uint16) if with_q else None
+    keys = {}
+    for i in range(T):
+        keys.setdefault((int(tok_seq[i]), int(tok_pos[i]) // POS_BLOCK), []).append(i)
+    for (b, blk), rows in keys.items():
+        a8, aqs, aw = _idx_query_block(cfg, b, blk)
+        sub = tok_pos[rows] % POS_BLOCK
+        q8[rows], qs[rows], w[rows] = a8[sub], aqs[sub], aw[sub]
+        if with_q:
+            q[rows] = _attn_query_block(cfg, b, blk)[sub]
+    return Queries(tok_seq, tok_pos, q8, qs, w, q)
+
+
+def _tie_table(cfg: Config):
+    rng = _rng(cfg.seed, 6)
+    base = rng.standard_normal((cfg.tie_vectors, cfg.idx_dim), dtype=np.float32)
+    return quantize_per_row(base)
+
+
+def make_cache(cfg: Config, with_kv: bool = True, queries: Optional[Queries] = None) -> PagedCache:
+    """Fill the paged caches for every sequence of ``cfg``.
+
+    Unused slots of each sequence's last page hold NaN poison, so a kernel that
+    reads past a sequence end produces NaN.  decode_128k needs the (decode)
+    queries to aim its planted keys; pass them or they are drawn here.
+    """
+    lens = seq_lens_of(cfg)
+    bt = block_table_of(cfg)
+    nb = int(sum((int(L) + PAGE - 1) // PAGE for L in lens))
+    rows = nb * PAGE
+    k8 = np.full((rows, cfg.idx_dim), POISON_FP8, np.uint8)
+    ks = np.full((rows,), np.nan, np.float32)
+    kv = np.full((rows, cfg.d_kv), POISON_BF16, np.uint16) if with_kv else None
+    tie = _tie_table(cfg) if cfg.tie_vectors else None
+    for b, L in enumerate(lens):
+        L = int(L)
+        for blk in range((L + PAGE - 1) // PAGE):
+            n = min(PAGE, L - blk * PAGE)
+            r0 = int(bt[b, blk]) * PAGE
+            rng = _rng(cfg.seed, 1, b, blk)
+            if tie is not None:
+                pick = rng.integers(0, cfg.tie_vectors, size=PAGE)[:n]
+                k8[r0:r0 + n] = tie[0][pick]
+                ks[r0:r0 + n] = tie[1][pick]
+            else:
+                kf = rng.standard_normal((PAGE, cfg.idx_dim), dtype=np.float32)[:n]
+                k8[r0:r0 + n], ks[r0:r0 + n] = quantize_per_row(kf)
+            if with_kv:
+                rv = _rng(cfg.seed, 2, b, blk)
+                kv[r0:r0 + n] = to_bf16_bits(
+                    rv.standard_normal((PAGE, cfg.d_kv), dtype=np.float32)[:n])
+    cache = PagedCache(k8, ks, kv, bt, lens.astype(np.int32))
+    if cfg.planted:
+        if queries is None:
+            queries = decode_queries(cfg, with_q=False)
+        plant_keys(cfg, cache, queries)
+    return cache
+
+
+def planted_positions(cfg: Config, b: int, L: int) -> np.ndarray:
+    """16 distinct positions in [0, L-2]; the first 4 inside the first 10% of context."""
+    rng = _rng(cfg.seed, 5, b)
+    n_early = cfg.planted // 4
+    early = rng.choice(max(1, L // 10), size=n_early, replace=False)
+    rest_pool = np.setdiff1d(np.arange(0, L - 1), early, assume_unique=False)
+    rest = rng.choice(rest_pool, size=cfg.planted - n_early, replace=False)
+    return np.sort(np.concatenate([early, rest])).astype(np.int64)
+
+
+def plant_keys(cfg: Config, cache: PagedCache, qs: Queries) -> None:
+    """Overwrite 16 keys per sequence with k = 3*sqrt(D_I)*u/|u| + 0.1*N(0,1),
+    u = sum_j max(w_j, 0) * qhat_j (the decode query's positively weighted heads)."""
+    for i in range(qs.n_tokens):
+        b = int(qs.tok_seq[i])
+        L = int(cache.seq_lens[b])
+        qhat = e4m3_values_torch(qs.q8[i]).astype(np.float64) * float(qs.q_scale[i])
+        u = (np.maximum(qs.w[i].astype(np.float64), 0)[:, None] * qhat).sum(0)
+        u /= np.linalg.norm(u)
+        pos = planted_positions(cfg, b, L)
+        noise = _rng(cfg.seed, 5, b, 1).standard_normal((pos.size, cfg.idx_dim))
+        kf = (3.0 * math.sqrt(cfg.idx_dim) * u[None, :] + 0.1 * noise).astype(np.float32)
+        rows = cache.phys_row(b, pos)
+        cache.k8[rows], cache.k_scale[rows] = quantize_per_row(kf)
+
+
+def decode_queries(cfg: Config, with_q: bool = True) -> Queries:
+    """One query per sequence at position L_b - 1 (tiny: positions 508..511)."""
+    lens = seq_lens_of(cfg)
+    if cfg.queries == "tail4":
+        L = int(lens[0])
+        return make_queries(cfg, [0] * 4, [L - 4, L - 3, L - 2, L - 1], with_q)
+    return make_queries(cfg, np.arange(cfg.batch), lens - 1, with_q)
+
+
+def prefill_queries(cfg: Config, chunk: int = 0, with_q: bool = True,
+                    positions: Optional[np.ndarray] = None) -> Queries:
+    """Causal prefill tokens.
+
+    prefill_16k: all 16384 positions of sequence 0 (or ``positions``).
+    chunked_64k: chunk ``chunk`` of every sequence, sequence-major
+    (positions chunk*4096 .. chunk*4096+4095 of sequence 0, then of sequence 1).
+    """
+    lens = seq_lens_of(cfg)
+    if cfg.chunk:
+        c0 = chunk * cfg.chunk
+        pos = np.arange(c0, c0 + cfg.chunk) if positions is None else np.asarray(positions)
+        seqs = np.repeat(np.arange(cfg.batch), pos.size)
+        return make_queries(cfg, seqs, np.tile(pos, cfg.batch), with_q)
+    pos = np.arange(int(lens[0])) if positions is None else np.asarray(positions)
+    return make_queries(cfg, np.zeros(pos.size, np.int32), pos, with_q)
+
+
+def make(name: str, with_kv: bool = True, with_q: bool = True, chunk: int = 0):
+    """(config, cache, queries) for the named workload's standard call."""
+    cfg = CONFIGS[name]
+    if cfg.queries == "prefill":
+        qs = prefill_queries(cfg, chunk=chunk, with_q=with_q)
+        cache = make_cache(cfg, with_kv=with_kv)
+    else:
+        qs = decode_queries(cfg, with_q=with_q)
+        cache = make_cache(cfg, with_kv=with_kv, queries=qs)
+    return cfg, cache, qs

@@ -1,0 +1,457 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each check compares the oracle with one of: the format definitions (golden code
+points), a worked example done by hand, brute force with an independent decoder
+(torch's FP8/BF16 casts) on tiny inputs, library special cases (torch's float64
+scaled_dot_product_attention, scipy's logsumexp, Python's sorted), closed forms
+and invariants that the DSA definition implies.  ``test_pins_catch_mutations``
+plants plausible mistakes in copies of the oracle and shows a pin fails for each.
+"""
+
+import math
+import os
+import types
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import dsa_ref as R
+from sparse_attention_long_03_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def torch_e4m3(b):
+    t = torch.from_numpy(np.ascontiguousarray(b, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def torch_bf16(u):
+    t = torch.from_numpy(np.ascontiguousarray(u, dtype=np.uint16).view(np.int16)).view(torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+def tiny_cache(rng, n_seq=2, lens=(70, 130), d_i=8, d_kv=24, h_i=3):
+    """A small random paged cache with a shuffled block table (several pages, ragged tail)."""
+    nblk = [(L + 63) // 64 for L in lens]
+    perm = rng.permutation(sum(nblk))
+    bt = np.full((n_seq, max(nblk)), -1, np.int32)
+    o = 0
+    for b, n in enumerate(nblk):
+        bt[b, :n] = perm[o:o + n]
+        o += n
+    rows = sum(nblk) * 64
+    k8, ks = W.quantize_per_row(rng.standard_normal((rows, d_i)).astype(np.float32))
+    kv = W.to_bf16_bits(rng.standard_normal((rows, d_kv)).astype(np.float32))
+    return types.SimpleNamespace(k8=k8, k_scale=ks, kv=kv, block_table=bt,
+                                 seq_lens=np.asarray(lens, np.int32), page=64)
+
+
+def tiny_query(rng, h_i=3, d_i=8, h=4, d_kv=24):
+    q8, qs = W.quantize_per_row(rng.standard_normal((1, h_i * d_i)).astype(np.float32))
+    w = rng.standard_normal(h_i).astype(np.float32)
+    q = W.to_bf16_bits(rng.standard_normal((h, d_kv)).astype(np.float32))
+    return q8.reshape(h_i, d_i), float(qs[0]), w, q
+
+
+# ----------------------------------------------------------------------------- formats
+
+def test_e4m3_exhaustive_matches_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    mine, ref = R.decode_e4m3(codes), torch_e4m3(codes)
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    assert np.isnan(mine).sum() == 2  # 0x7F and 0xFF only
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+    assert np.array_equal(np.signbit(mine[ok]), np.signbit(ref[ok]))
+
+
+def test_e4m3_golden_points():
+    for line in open(os.path.join(GOLDEN, "e4m3_points.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        code, val = line.split()
+        got = float(R.decode_e4m3(np.uint8(int(code, 16))))
+        if val == "nan":
+            assert math.isnan(got)
+        else:
+            assert got == float(val) and math.copysign(1, got) == math.copysign(1, float(val))
+
+
+def test_bf16_matches_torch():
+    rng = np.random.default_rng(0)
+    u = rng.integers(0, 1 << 16, size=200000, dtype=np.uint32).astype(np.uint16)
+    u = u[~(((u >> 7) & 0xFF) == 0xFF)]  # finite patterns
+    assert np.array_equal(R.decode_bf16(u), torch_bf16(u))
+    assert R.decode_bf16(np.uint16(0x3F80)) == 1.0
+    assert R.decode_bf16(np.uint16(0xC000)) == -2.0
+    assert R.decode_bf16(np.uint16(0x7F80)) == np.inf
+
+
+# ----------------------------------------------------------------------------- indexer
+
+def test_indexer_hand_example():
+    q, w, keys, expect, top2 = None, None, [], None, None
+    for line in open(os.path.join(GOLDEN, "indexer_hand_example.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        f = line.split()
+        if f[0] == "q":
+            q = np.array([int(x, 16) for x in f[1:]], np.uint8).reshape(2, 2)
+        elif f[0] == "w":
+            w = np.array([float(x) for x in f[1:]])
+        elif f[0] == "k":
+            keys.append(([int(f[1], 16), int(f[2], 16)], float(f[3])))
+        elif f[0] == "expect":
+            expect = np.array([float(x) for x in f[1:]])
+        elif f[0] == "top2":
+            top2 = [int(x) for x in f[1:]]
+    k8 = np.full((64, 2), 0x7F, np.uint8)
+    ks = np.full(64, np.nan, np.float32)
+    for s, (b, sc) in enumerate(keys):
+        k8[s], ks[s] = b, sc
+    bt = np.array([[0]], np.int32)
+    got = R.indexer_logits_row(k8, ks, bt, 0, 2, q, 1.0, w)
+    assert np.array_equal(got, expect)
+    assert list(R.topk_select(got, 2)) == top2
+
+
+def brute_force_logit(cache, b, s, q8_t, qs_t, w_t):
+    phys = int(cache.block_table[b][s // 64]) * 64 + s % 64
+    kh = torch_e4m3(cache.k8[phys]) * float(cache.k_scale[phys])
+    qh = torch_e4m3(q8_t) * float(qs_t)
+    acc = 0.0
+    for j in range(qh.shape[0]):
+        dot = 0.0
+        for d in range(qh.shape[1]):
+            dot += float(qh[j, d]) * float(kh[d])
+        acc += float(w_t[j]) * (dot if dot > 0 else 0.0)
+    return acc
+
+
+def check_indexer_brute_force(fn):
+    rng = np.random.default_rng(1)
+    c = tiny_cache(rng)
+    for b, pos in ((0, 69), (1, 100), (1, 129), (0, 0)):
+        q8, qs, w, _ = tiny_query(rng)
+        got = fn(c.k8, c.k_scale, c.block_table, b, pos, q8, qs, w)
+        assert got.shape == (pos + 1,)
+        ref = np.array([brute_force_logit(c, b, s, q8, qs, w) for s in range(pos + 1)])
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_indexer_brute_force():
+    check_indexer_brute_force(R.indexer_logits_row)
+
+
+def check_indexer_relu_closed_form(fn):
+    # one head, one dim: I[s] = w * max(0, q * k[s]); with q = 1 (0x38), w = 0.75
+    k8 = np.array([[0x40], [0xC0], [0x38], [0xB8], [0x00]] + [[0x7F]] * 59, np.uint8)
+    ks = np.array([1.0, 1.0, 3.0, 3.0, 1.0] + [np.nan] * 59, np.float32)
+    got = fn(k8, ks, np.array([[0]], np.int32), 0, 4, np.array([[0x38]], np.uint8), 1.0,
+             np.array([0.75]))
+    np.testing.assert_array_equal(got, [1.5, 0.0, 2.25, 0.0, 0.0])
+
+
+def test_indexer_relu_closed_form():
+    check_indexer_relu_closed_form(R.indexer_logits_row)
+
+
+def test_indexer_scales_and_weights():
+    rng = np.random.default_rng(2)
+    c = tiny_cache(rng)
+    q8, qs, w, _ = tiny_query(rng)
+    base = R.indexer_logits_row(c.k8, c.k_scale, c.block_table, 1, 120, q8, qs, w)
+    # positive homogeneity in each scale (ReLU commutes with positive scaling)
+    np.testing.assert_allclose(
+        R.indexer_logits_row(c.k8, c.k_scale, c.block_table, 1, 120, q8, 2 * qs, w), 2 * base,
+        rtol=1e-12)
+    ks2 = c.k_scale.copy()
+    rows = R.logical_rows(c.block_table, 1, 121)
+    ks2[rows[7]] *= 3
+    got = R.indexer_logits_row(c.k8, ks2, c.block_table, 1, 120, q8, qs, w)
+    exp = base.copy()
+    exp[7] *= 3
+    np.testing.assert_allclose(got, exp, rtol=1e-12)
+    # linear in w; w >= 0 gives I >= 0
+    w2 = rng.standard_normal(w.shape)
+    a = R.indexer_logits_row(c.k8, c.k_scale, c.block_table, 1, 120, q8, qs, w2)
+    ab = R.indexer_logits_row(c.k8, c.k_scale, c.block_table, 1, 120, q8, qs, w + w2)
+    np.testing.assert_allclose(ab, base + a, rtol=1e-9, atol=1e-9)
+    pos = R.indexer_logits_row(c.k8, c.k_scale, c.block_table, 1, 120, q8, qs, np.abs(w))
+    assert (pos >= 0).all() and (pos > 0).any()
+
+
+def test_indexer_block_table_permutation_invariance():
+    rng = np.random.default_rng(3)
+    c = tiny_cache(rng, n_seq=1, lens=(200,))
+    q8, qs, w, _ = tiny_query(rng)
+    ref = R.indexer_logits_row(c.k8, c.k_scale, c.block_table, 0, 199, q8, qs, w)
+    # move every page to a different physical block
+    nb = c.block_table.shape[1]
+    newpos = rng.permutation(nb)
+    k8 = np.empty_like(c.k8)
+    ks = np.empty_like(c.k_scale)
+    bt = np.empty_like(c.block_table)
+    for lb in range(nb):
+        old, new = int(c.block_table[0, lb]), int(newpos[lb])
+        k8[new * 64:(new + 1) * 64] = c.k8[old * 64:(old + 1) * 64]
+        ks[new * 64:(new + 1) * 64] = c.k_scale[old * 64:(old + 1) * 64]
+        bt[0, lb] = new
+    got = R.indexer_logits_row(k8, ks, bt, 0, 199, q8, qs, w)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_indexer_never_reads_past_position():
+    # poison (NaN) everywhere after the query position: the row must stay finite
+    rng = np.random.default_rng(4)
+    c = tiny_cache(rng, n_seq=1, lens=(128,))
+    q8, qs, w, _ = tiny_query(rng)
+    rows = R.logical_rows(c.block_table, 0, 128)
+    c.k8[rows[51:]] = 0x7F
+    c.k_scale[rows[51:]] = np.nan
+    assert np.isfinite(R.indexer_logits_row(c.k8, c.k_scale, c.block_table, 0, 50, q8, qs, w)).all()
+
+
+# ----------------------------------------------------------------------------- top-k
+
+def check_topk_vs_sorted(fn):
+    rng = np.random.default_rng(5)
+    for n, k in ((1, 4), (7, 3), (40, 40), (50, 8), (300, 32), (301, 300)):
+        row = rng.integers(-4, 5, size=n).astype(np.float64) * 0.5  # many ties
+        ref = sorted(sorted(range(n), key=lambda s: (-row[s], s))[:min(k, n)])
+        assert list(fn(row, k)) == ref
+        row2 = rng.standard_normal(n)
+        ref2 = sorted(sorted(range(n), key=lambda s: (-row2[s], s))[:min(k, n)])
+        assert list(fn(row2, k)) == ref2
+
+
+def test_topk_vs_sorted():
+    check_topk_vs_sorted(R.topk_select)
+
+
+def test_topk_fewer_than_k_selects_all():
+    assert list(R.topk_select(np.array([3.0, -1.0, 2.0]), 2048)) == [0, 1, 2]
+    assert R.kth_value(np.array([3.0, -1.0, 2.0]), 2) == 2.0
+
+
+# ----------------------------------------------------------------------------- attention
+
+def attn_case(rng, n_keys=150, h=4, d_kv=24, d_v=16):
+    c = tiny_cache(rng, n_seq=1, lens=(n_keys,), d_kv=d_kv)
+    _, _, _, q = tiny_query(rng, h=h, d_kv=d_kv)
+    return c, q
+
+
+def check_attention_dense_equivalence(fn):
+    """k >= L: the sparse path is standard causal attention over all preceding tokens
+    (torch float64 SDPA, latent rows broadcast to every head = MQA)."""
+    rng = np.random.default_rng(6)
+    c, q = attn_case(rng)
+    scale, d_v, pos = 0.3, 16, 149
+    out, lse = fn(c.kv, c.block_table, 0, q, np.arange(pos + 1), scale, d_v)
+    rows = R.logical_rows(c.block_table, 0, pos + 1)
+    kv = torch.from_numpy(torch_bf16(c.kv[rows]))  # [n, D]
+    qt = torch.from_numpy(torch_bf16(q))  # [H, D]
+    H = qt.shape[0]
+    ref = F.scaled_dot_product_attention(qt[None, :, None, :], kv[None, None].expand(1, H, -1, -1),
+                                         kv[None, None, :, :d_v].expand(1, H, -1, -1), scale=scale)
+    np.testing.assert_allclose(out, ref[0, :, 0].numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_attention_dense_equivalence():
+    check_attention_dense_equivalence(R.sparse_mla_attn_token)
+
+
+def test_attention_dense_causal_prefill():
+    """Every query position of a 100-token prefill with k >= 100 equals is_causal SDPA."""
+    rng = np.random.default_rng(7)
+    c = tiny_cache(rng, n_seq=1, lens=(100,))
+    H, D, dv, scale = 3, 24, 16, 0.2
+    qs = W.to_bf16_bits(rng.standard_normal((100, H, D)).astype(np.float32))
+    rows = R.logical_rows(c.block_table, 0, 100)
+    kv = torch.from_numpy(torch_bf16(c.kv[rows]))
+    qt = torch.from_numpy(torch_bf16(qs)).permute(1, 0, 2)[None]  # [1,H,T,D]
+    ref = F.scaled_dot_product_attention(qt, kv[None, None].expand(1, H, -1, -1),
+                                         kv[None, None, :, :dv].expand(1, H, -1, -1),
+                                         is_causal=True, scale=scale)[0].permute(1, 0, 2).numpy()
+    for t in (0, 1, 37, 99):
+        sel = R.topk_select(np.zeros(t + 1), 2048)
+        out, _ = R.sparse_mla_attn_token(c.kv, c.block_table, 0, qs[t], sel, scale, dv)
+        np.testing.assert_allclose(out, ref[t], rtol=1e-12, atol=1e-13)
+
+
+def check_attention_single_and_two_keys(fn):
+    rng = np.random.default_rng(8)
+    c, q = attn_case(rng)
+    scale, d_v = 0.25, 16
+    rows = R.logical_rows(c.block_table, 0, 150)
+    kvh = torch_bf16(c.kv[rows])
+    qh = torch_bf16(q)
+    out, lse = fn(c.kv, c.block_table, 0, q, [42], scale, d_v)
+    np.testing.assert_array_equal(out, np.broadcast_to(kvh[42, :d_v], out.shape))
+    np.testing.assert_allclose(lse, scale * qh @ kvh[42], rtol=1e-13)
+    out, lse = fn(c.kv, c.block_table, 0, q, [3, 120], scale, d_v)
+    z1, z2 = scale * qh @ kvh[3], scale * qh @ kvh[120]
+    p1 = 1.0 / (1.0 + np.exp(z2 - z1))
+    ref = p1[:, None] * kvh[3, :d_v] + (1 - p1)[:, None] * kvh[120, :d_v]
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, np.logaddexp(z1, z2), rtol=1e-13)
+
+
+def test_attention_single_and_two_keys():
+    check_attention_single_and_two_keys(R.sparse_mla_attn_token)
+
+
+def test_attention_softmax_rows_sum_to_one():
+    rng = np.random.default_rng(9)
+    c, q = attn_case(rng)
+    sel = rng.choice(150, size=60, replace=False)
+    p = R.softmax_weights(c.kv, c.block_table, 0, q, sel, 0.4)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=1e-14)
+    # constant value rows -> the output is that constant
+    kv = c.kv.copy()
+    kv[:, :16] = 0x3FC0  # bf16 1.5
+    out, _ = R.sparse_mla_attn_token(kv, c.block_table, 0, q, sel, 0.4, 16)
+    np.testing.assert_allclose(out, 1.5, rtol=1e-14)
+
+
+def test_attention_order_invariance_lse_and_mqa():
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(10)
+    c, q = attn_case(rng)
+    sel = rng.choice(150, size=64, replace=False)
+    o1, l1 = R.sparse_mla_attn_token(c.kv, c.block_table, 0, q, sel, 0.3, 16)
+    o2, l2 = R.sparse_mla_attn_token(c.kv, c.block_table, 0, q, sel[::-1], 0.3, 16)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-14)
+    rows = R.logical_rows(c.block_table, 0, 150)
+    z = 0.3 * torch_bf16(q) @ torch_bf16(c.kv[rows][sel]).T
+    np.testing.assert_allclose(l1, logsumexp(z, axis=1), rtol=1e-13)
+    qsame = np.repeat(q[:1], q.shape[0], axis=0)
+    o3, _ = R.sparse_mla_attn_token(c.kv, c.block_table, 0, qsame, sel, 0.3, 16)
+    assert np.array_equal(o3, np.repeat(o3[:1], q.shape[0], axis=0))
+
+
+# ----------------------------------------------------------------------------- work counts
+
+def test_work_counts_quadratic_vs_linear():
+    k = 2048
+    for L in (1000, 2048, 16384, 65536):
+        ind, att = R.work_counts(np.arange(L), k)
+        assert ind == L * (L + 1) // 2
+        assert att == (L * (L + 1) // 2 if L <= k else k * (k + 1) // 2 + (L - k) * k)
+    # doubling L quadruples the indexer work but only doubles the attention work (L >> k)
+    i1, a1 = R.work_counts(np.arange(1 << 17), k)
+    i2, a2 = R.work_counts(np.arange(1 << 18), k)
+    assert 3.99 < i2 / i1 < 4.01 and 1.99 < a2 / a1 < 2.02
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def test_tiny_workload_end_to_end_finite():
+    cfg, cache, qs = W.make("tiny")
+    for t in range(qs.n_tokens):
+        logits, sel, out, lse = R.dsa_forward_token(cache, qs, t, cfg.topk, cfg.scale, cfg.d_v)
+        assert logits.shape == (int(qs.tok_pos[t]) + 1,) and np.isfinite(logits).all()
+        assert sel.shape == (cfg.topk,) and np.isfinite(out).all() and np.isfinite(lse).all()
+
+
+@pytest.mark.slow
+def test_planted_keys_are_selected():
+    """decode_128k: every planted key (aimed along the query) is in the oracle's top-k."""
+    cfg = W.CONFIGS["decode_128k"]
+    qs = W.decode_queries(cfg, with_q=False)
+    cache = W.make_cache(cfg, with_kv=False, queries=qs)
+    for t in range(qs.n_tokens):
+        b = int(qs.tok_seq[t])
+        row = R.indexer_logits_row(cache.k8, cache.k_scale, cache.block_table, b,
+                                   int(qs.tok_pos[t]), qs.q8[t], qs.q_scale[t], qs.w[t])
+        sel = set(R.topk_select(row, cfg.topk).tolist())
+        planted = W.planted_positions(cfg, b, int(cache.seq_lens[b]))
+        assert set(planted.tolist()) <= sel
+        assert (planted < int(cache.seq_lens[b]) // 10).sum() >= 4
+
+
+# ----------------------------------------------------------------------------- mutations
+
+def _mutants():
+    """Plausible mistakes, each planted in a copy of one oracle function."""
+
+    def no_kscale(k8, ks, bt, b, pos, q8, qs, w, page=64):
+        rows = R.logical_rows(bt, b, pos + 1, page)
+        khat = R.decode_e4m3(k8[rows])
+        return np.maximum(khat @ (R.decode_e4m3(q8) * qs).T, 0) @ w
+
+    def relu_after_sum(k8, ks, bt, b, pos, q8, qs, w, page=64):
+        rows = R.logical_rows(bt, b, pos + 1, page)
+        khat = R.decode_e4m3(k8[rows]) * np.asarray(ks, np.float64)[rows, None]
+        return np.maximum((khat @ (R.decode_e4m3(q8) * qs).T) @ w, 0)
+
+    def exclusive_causal(k8, ks, bt, b, pos, q8, qs, w, page=64):
+        return R.indexer_logits_row(k8, ks, bt, b, max(pos - 1, 0), q8, qs, w, page)
+
+    def block_index_swapped(k8, ks, bt, b, pos, q8, qs, w, page=64):
+        s = np.arange(pos + 1)
+        rows = np.asarray(bt)[b, s % page].astype(np.int64) * page + s // page
+        rows = np.clip(rows, 0, k8.shape[0] - 1)
+        khat = R.decode_e4m3(k8[rows]) * np.asarray(ks, np.float64)[rows, None]
+        return np.maximum(khat @ (R.decode_e4m3(q8) * qs).T, 0) @ w
+
+    def topk_ties_large_s(row, k):
+        row = np.asarray(row, np.float64)
+        order = np.lexsort((-np.arange(row.shape[0]), -row))
+        return np.sort(order[:min(k, row.shape[0])])
+
+    def topk_smallest(row, k):
+        return np.sort(np.argsort(np.asarray(row), kind="stable")[:min(k, len(row))])
+
+    def attn_no_scale(kv, bt, b, q, sel, scale, d_v, page=64):
+        return R.sparse_mla_attn_token(kv, bt, b, q, sel, 1.0, d_v, page)
+
+    def attn_rope_dropped(kv, bt, b, q, sel, scale, d_v, page=64):
+        kv2 = np.asarray(kv).copy()
+        kv2[:, d_v:] = 0
+        q2 = np.asarray(q).copy()
+        q2[:, d_v:] = 0
+        return R.sparse_mla_attn_token(kv2, bt, b, q2, sel, scale, d_v, page)
+
+    def attn_value_from_tail(kv, bt, b, q, sel, scale, d_v, page=64):
+        out, lse = R.sparse_mla_attn_token(kv, bt, b, q, sel, scale, np.asarray(kv).shape[1], page)
+        return out[:, -d_v:], lse
+
+    def attn_unnormalised(kv, bt, b, q, sel, scale, d_v, page=64):
+        sel = np.asarray(sel)
+        rows = np.asarray(bt)[b, sel // page].astype(np.int64) * page + sel % page
+        kvh = R.decode_bf16(np.asarray(kv)[rows])
+        z = scale * (R.decode_bf16(q) @ kvh.T)
+        e = np.exp(z - z.max(1, keepdims=True))
+        return e @ kvh[:, :d_v], (z.max(1) + np.log(e.sum(1)))
+
+    return [
+        ("indexer", no_kscale), ("indexer", relu_after_sum), ("indexer", exclusive_causal),
+        ("indexer", block_index_swapped), ("topk", topk_ties_large_s), ("topk", topk_smallest),
+        ("attn", attn_no_scale), ("attn", attn_rope_dropped), ("attn", attn_value_from_tail),
+        ("attn", attn_unnormalised),
+    ]
+
+
+PIN_CHECKS = {
+    "indexer": [check_indexer_brute_force, check_indexer_relu_closed_form],
+    "topk": [check_topk_vs_sorted],
+    "attn": [check_attention_dense_equivalence, check_attention_single_and_two_keys],
+}
+
+
+@pytest.mark.parametrize("kind,mutant", _mutants(), ids=lambda x: getattr(x, "__name__", x))
+def test_pins_catch_mutations(kind, mutant):
+    caught = 0
+    for check in PIN_CHECKS[kind]:
+        try:
+            check(mutant)
+        except (AssertionError, ValueError, IndexError):
+            caught += 1
+    assert caught >= 1, f"no pin catches mutant {mutant.__name__}"
