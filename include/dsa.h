@@ -1,0 +1,148 @@
+/*
+ * dsa.h — C ABI of libdsa.so, the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * The path (pages "DeepSeek V3.2-Exp Cuts Prolonged-Context Costs With DeepSeek Sparse
+ * Attention (DSA) ..." and its Spanish translation, section "FP8 index -> top-k selection
+ * -> sparse core attention"):
+ *   (1) lightning indexer   I[t,s] = sum_j w[t,j] * ReLU(qhat[t,j,:] . khat[s,:]), s <= pos(t)
+ *   (2) top-k selection     the k (= 2048) largest I[t,s] per query token
+ *   (3) sparse attention    softmax attention over only the selected latent rows, MLA in
+ *                           MQA mode: all query heads share each 576-wide latent row
+ *                           (512 latent + 64 rope); the value is the 512-wide latent.
+ * Keys and latent rows live in a paged cache of 64-token pages ("DeepSeek V3.2-Exp: Sparse
+ * Attention, Long Context, and Cheaper API", section "Quick guide to run it locally":
+ * --page-size 64; section "Open kernels and ecosystem support": paged indexer kernels).
+ *
+ * Conventions (all entry points):
+ *   - Every pointer argument named "device" is CUDA device memory owned by the caller;
+ *     the library never allocates, frees or keeps a pointer after the call returns
+ *     (except the stream-ordered work it enqueued).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Calls are asynchronous: they validate, enqueue kernels and return.
+ *   - The return value reports host-side validation and launch errors only.  Errors
+ *     found by the kernels (a block-table entry or index out of range, a bounded wait
+ *     that gave up) are recorded in a per-device status word that
+ *     dsa_read_device_status() returns and clears.  A kernel that finds a bad entry
+ *     skips the access it would have made and writes NaN (floats) or -1 (indices) there.
+ *   - FP8 is OCP e4m3 ("fn": bias 7, no infinities, max 448) stored as bytes; BF16 is
+ *     stored as its 16-bit pattern (the upper half of an IEEE fp32).
+ *   - Supported shapes: page_size 64; idx_dim in {32, 64, 128}; n_idx_heads in 1..64;
+ *     n_heads in 1..128; d_kv a multiple of 16 in 16..576; d_v a multiple of 64,
+ *     64 <= d_v <= min(d_kv, 512); 1 <= k <= 2048.  Anything else: DSA_ERR_UNSUPPORTED.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent arguments   */
+  DSA_ERR_UNSUPPORTED = 2,  /* valid but outside the supported shapes listed above  */
+  DSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than the *_workspace_size */
+  DSA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed                  */
+  DSA_ERR_BAD_INDEX = 5,    /* (device) block-table entry or index out of range      */
+  DSA_ERR_TIMEOUT = 6       /* (device) a bounded in-kernel wait gave up             */
+} dsa_status;
+
+/* Paged caches, one row per cached token.  Token s of sequence b lives in physical row
+ *   block_table[b * max_blocks_per_seq + s / page_size] * page_size + s % page_size.   */
+typedef struct {
+  const uint8_t* k8;          /* device [num_blocks*page_size, idx_dim]  e4m3 index keys   */
+  const float* k_scale;       /* device [num_blocks*page_size]           per-token scale   */
+  const uint16_t* kv;         /* device [num_blocks*page_size, d_kv]     bf16 latent rows  */
+  const int32_t* block_table; /* device [batch, max_blocks_per_seq]      physical blocks   */
+  int32_t batch;              /* number of sequences                                       */
+  int32_t max_blocks_per_seq; /* row stride of block_table                                 */
+  int32_t num_blocks;         /* physical blocks in the caches (bounds for block_table)    */
+  int32_t page_size;          /* tokens per block; must be 64                              */
+  int32_t idx_dim;            /* D_I: bytes per index key                                  */
+  int32_t d_kv;               /* latent row width (latent + rope), bf16 elements           */
+} dsa_paged_cache;
+
+/* The query tokens of one call, flattened over sequences.  Query t attends to tokens
+ * 0..tok_pos[t] of sequence tok_seq[t] (itself included).  Tokens of one sequence should be
+ * contiguous and in increasing position: the indexer then shares each key tile among up
+ * to four of them (any order is still correct, only slower).                               */
+typedef struct {
+  int32_t n_tokens;        /* T >= 0                                                     */
+  const int32_t* tok_seq;  /* device [T]  sequence of each token, 0 <= tok_seq < batch   */
+  const int32_t* tok_pos;  /* device [T]  position of each token, 0 <= tok_pos <= max_pos */
+  int32_t max_pos;         /* host: an upper bound on every tok_pos (sizes grids/buffers) */
+} dsa_queries;
+
+/* (1) Lightning indexer (FP8 tcgen05 MMA over the paged e4m3 key cache).
+ * q8       device [T, n_idx_heads, idx_dim]  e4m3 indexer queries
+ * q_scale  device [T]                        per-token scale of q8 (> 0)
+ * w        device [T, n_idx_heads]           fp32 head weights
+ * logits   device [T, ld_logits] fp32: row t gets I[t,s] for s = 0..tok_pos[t];
+ *          entries past tok_pos[t] are not written.  ld_logits >= max_pos + 1.
+ * workspace: device, >= dsa_indexer_workspace_size(n_tokens) bytes, 256-byte aligned.   */
+DSA_API dsa_status dsa_indexer_logits(const dsa_paged_cache* cache, const dsa_queries* queries,
+                              const uint8_t* q8, const float* q_scale, const float* w,
+                              int32_t n_idx_heads, float* logits, int64_t ld_logits,
+                              void* workspace, size_t workspace_bytes, void* stream);
+DSA_API size_t dsa_indexer_workspace_size(int32_t n_tokens);
+
+/* (2) Per-row top-k by radix select (no sort) over logits[t, 0..tok_pos[t]].
+ * idx  device [T, k] int32: the logical positions of the min(k, tok_pos[t]+1) largest
+ *      logits of row t (equal values: the smaller position first), -1 in unused slots.
+ *      The order inside a row is unspecified but deterministic (same input, same output).
+ * workspace: device, >= dsa_topk_workspace_size(n_tokens, max_pos, k) bytes.            */
+DSA_API dsa_status dsa_topk(const float* logits, int64_t ld_logits, const dsa_queries* queries,
+                    int32_t k, int32_t* idx, void* workspace, size_t workspace_bytes,
+                    void* stream);
+DSA_API size_t dsa_topk_workspace_size(int32_t n_tokens, int32_t max_pos, int32_t k);
+
+/* (3) Sparse MLA attention, MQA mode (BF16 tcgen05 MMA, fp32 online softmax).
+ * q    device [T, n_heads, d_kv] bf16 queries
+ * idx  device [T, k] int32 logical positions (-1 = empty slot, skipped); every
+ *      non-negative entry must be <= tok_pos[t]
+ * out  device [T, n_heads, d_v] bf16:  sum_s softmax_s(scale * q.kv[s]) * kv[s, :d_v]
+ * lse  device [T, n_heads] fp32 log-sum-exp of scale*q.kv over the selected rows, or NULL
+ * A row with no selected entry gets out = 0 and lse = -inf.
+ * workspace: device, >= dsa_attn_workspace_size(n_tokens, n_heads, d_v, k) bytes.      */
+DSA_API dsa_status dsa_sparse_mla_attn(const dsa_paged_cache* cache, const dsa_queries* queries,
+                               const uint16_t* q, int32_t n_heads, int32_t d_v, float scale,
+                               const int32_t* idx, int32_t k, uint16_t* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream);
+DSA_API size_t dsa_attn_workspace_size(int32_t n_tokens, int32_t n_heads, int32_t d_v, int32_t k);
+
+/* (1)+(2)+(3) in one call; the logits and selected indices live in the workspace
+ * (idx_out, if not NULL, receives a copy of the selection, device [T, k] int32).
+ * A chunked prefill is a sequence of calls, each over one chunk's tokens, against the
+ * cache prefix that already holds the chunk's own keys and latent rows.                  */
+DSA_API dsa_status dsa_forward(const dsa_paged_cache* cache, const dsa_queries* queries,
+                       const uint8_t* q8, const float* q_scale, const float* w,
+                       int32_t n_idx_heads, const uint16_t* q, int32_t n_heads, int32_t d_v,
+                       float scale, int32_t k, uint16_t* out, float* lse, int32_t* idx_out,
+                       void* workspace, size_t workspace_bytes, void* stream);
+DSA_API size_t dsa_forward_workspace_size(int32_t n_tokens, int32_t max_pos, int32_t k,
+                                  int32_t n_heads, int32_t d_v);
+
+/* Waits for `stream`, then returns and clears the device status word of the current
+ * device (DSA_OK, DSA_ERR_BAD_INDEX or DSA_ERR_TIMEOUT; DSA_ERR_CUDA if the wait failed). */
+DSA_API dsa_status dsa_read_device_status(void* stream);
+
+/* Number of kernel launches the library has enqueued in this process (all devices). */
+DSA_API int64_t dsa_launch_count(void);
+
+DSA_API const char* dsa_status_string(dsa_status status);
+DSA_API int32_t dsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

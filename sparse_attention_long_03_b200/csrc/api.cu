@@ -1,0 +1,241 @@
+// C ABI of libdsa.so: argument validation, workspace layout and kernel launches.
+// Every entry point only enqueues work on the caller's stream; nothing here allocates.
+#include <atomic>
+#include <cstring>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+__device__ uint32_t g_status = 0;
+
+static std::atomic<int64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+int num_sms() {
+  static int cached[64];
+  static bool init[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!init[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+    init[dev] = true;
+  }
+  return cached[dev];
+}
+
+cudaError_t read_and_clear_status(cudaStream_t stream, uint32_t* out) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  uint32_t v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof(v));
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+  *out = v;
+  return e;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+static bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+static dsa_status check_cache(const dsa_paged_cache* c, bool need_keys, bool need_kv) {
+  if (!c || !c->block_table) return DSA_ERR_INVALID_ARG;
+  if (c->batch <= 0 || c->max_blocks_per_seq <= 0 || c->num_blocks <= 0) return DSA_ERR_INVALID_ARG;
+  if (c->page_size != kPage) return DSA_ERR_UNSUPPORTED;
+  if (need_keys) {
+    if (!c->k8 || !c->k_scale) return DSA_ERR_INVALID_ARG;
+    if (c->idx_dim != 32 && c->idx_dim != 64 && c->idx_dim != 128) return DSA_ERR_UNSUPPORTED;
+    if (!aligned(c->k8, 16) || !aligned(c->k_scale, 4)) return DSA_ERR_INVALID_ARG;
+  }
+  if (need_kv) {
+    if (!c->kv) return DSA_ERR_INVALID_ARG;
+    if (c->d_kv < 16 || c->d_kv > 576 || c->d_kv % 16) return DSA_ERR_UNSUPPORTED;
+    if (!aligned(c->kv, 16)) return DSA_ERR_INVALID_ARG;
+  }
+  return DSA_OK;
+}
+
+static dsa_status check_queries(const dsa_queries* q) {
+  if (!q || q->n_tokens < 0 || q->max_pos < 0) return DSA_ERR_INVALID_ARG;
+  if (q->n_tokens > 0 && (!q->tok_seq || !q->tok_pos)) return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+static dsa_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return DSA_OK;
+  if (e == cudaErrorNotSupported) return DSA_ERR_UNSUPPORTED;
+  cudaGetLastError();
+  return DSA_ERR_CUDA;
+}
+
+static dsa_status check_attn_shape(int32_t n_heads, int32_t d_kv, int32_t d_v, int32_t k) {
+  if (n_heads < 1 || n_heads > 128) return DSA_ERR_UNSUPPORTED;
+  if (d_v < 64 || d_v > 512 || d_v % 64 || d_v > d_kv) return DSA_ERR_UNSUPPORTED;
+  if (k < 1 || k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
+  // value chunks of the first CTA plus the rope chunks must fit its five chunk slots
+  const int nc = (d_kv + 63) / 64, nv = d_v / 64;
+  if ((nv + 1) / 2 + (nc - nv) > 5) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+// Forward workspace: [indexer plan][logits T x ld][idx T x k][attention partials]
+struct ForwardLayout {
+  size_t plan, logits, idx, attn, total;
+  int64_t ld;
+};
+static ForwardLayout forward_layout(int32_t T, int32_t max_pos, int32_t k, int32_t H,
+                                    int32_t d_v) {
+  ForwardLayout L;
+  L.ld = ((static_cast<int64_t>(max_pos) + 1 + 127) / 128) * 128;
+  L.plan = 0;
+  size_t off = align256(indexer_ws_bytes(T));
+  L.logits = off;
+  off += align256(static_cast<size_t>(T) * L.ld * 4);
+  L.idx = off;
+  off += align256(static_cast<size_t>(T) * k * 4);
+  L.attn = off;
+  off += align256(attn_ws_bytes(T, H, d_v, k));
+  L.total = off;
+  return L;
+}
+
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+int32_t dsa_abi_version(void) { return 1; }
+
+int64_t dsa_launch_count(void) { return g_launches.load(); }
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSA_ERR_WORKSPACE: return "workspace too small";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_BAD_INDEX: return "block-table entry or index out of range (device)";
+    case DSA_ERR_TIMEOUT: return "bounded in-kernel wait gave up (device)";
+  }
+  return "unknown status";
+}
+
+size_t dsa_indexer_workspace_size(int32_t n_tokens) { return indexer_ws_bytes(n_tokens); }
+
+size_t dsa_topk_workspace_size(int32_t n_tokens, int32_t max_pos, int32_t k) {
+  return topk_ws_bytes(n_tokens, max_pos, k);
+}
+
+size_t dsa_attn_workspace_size(int32_t n_tokens, int32_t n_heads, int32_t d_v, int32_t k) {
+  return attn_ws_bytes(n_tokens, n_heads, d_v, k);
+}
+
+size_t dsa_forward_workspace_size(int32_t n_tokens, int32_t max_pos, int32_t k, int32_t n_heads,
+                                  int32_t d_v) {
+  if (n_tokens < 0 || max_pos < 0) return 0;
+  return forward_layout(n_tokens, max_pos, k, n_heads, d_v).total;
+}
+
+dsa_status dsa_indexer_logits(const dsa_paged_cache* cache, const dsa_queries* queries,
+                              const uint8_t* q8, const float* q_scale, const float* w,
+                              int32_t n_idx_heads, float* logits, int64_t ld_logits,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status s = check_cache(cache, true, false);
+  if (s != DSA_OK) return s;
+  if ((s = check_queries(queries)) != DSA_OK) return s;
+  if (n_idx_heads < 1 || n_idx_heads > 64) return DSA_ERR_UNSUPPORTED;
+  if (queries->n_tokens == 0) return DSA_OK;
+  if (!q8 || !q_scale || !w || !logits) return DSA_ERR_INVALID_ARG;
+  if (!aligned(q8, 16) || !aligned(w, 4) || !aligned(logits, 4)) return DSA_ERR_INVALID_ARG;
+  if (ld_logits < static_cast<int64_t>(queries->max_pos) + 1) return DSA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < indexer_ws_bytes(queries->n_tokens) ||
+      !aligned(workspace, 256))
+    return DSA_ERR_WORKSPACE;
+  IndexerLaunch L{cache, queries, q8, q_scale, w, n_idx_heads, logits, ld_logits, workspace,
+                  static_cast<cudaStream_t>(stream)};
+  return cuda_status(launch_indexer(L));
+}
+
+dsa_status dsa_topk(const float* logits, int64_t ld_logits, const dsa_queries* queries, int32_t k,
+                    int32_t* idx, void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status s = check_queries(queries);
+  if (s != DSA_OK) return s;
+  if (k < 1 || k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
+  if (queries->n_tokens == 0) return DSA_OK;
+  if (!logits || !idx) return DSA_ERR_INVALID_ARG;
+  if (ld_logits < static_cast<int64_t>(queries->max_pos) + 1) return DSA_ERR_INVALID_ARG;
+  if (workspace_bytes < topk_ws_bytes(queries->n_tokens, queries->max_pos, k))
+    return DSA_ERR_WORKSPACE;
+  return cuda_status(launch_topk(logits, ld_logits, queries, k, idx, workspace,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_sparse_mla_attn(const dsa_paged_cache* cache, const dsa_queries* queries,
+                               const uint16_t* q, int32_t n_heads, int32_t d_v, float scale,
+                               const int32_t* idx, int32_t k, uint16_t* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status s = check_cache(cache, false, true);
+  if (s != DSA_OK) return s;
+  if ((s = check_queries(queries)) != DSA_OK) return s;
+  if ((s = check_attn_shape(n_heads, cache->d_kv, d_v, k)) != DSA_OK) return s;
+  if (!(scale > 0.f) || scale != scale) return DSA_ERR_INVALID_ARG;
+  if (queries->n_tokens == 0) return DSA_OK;
+  if (!q || !idx || !out) return DSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16)) return DSA_ERR_INVALID_ARG;
+  const size_t need = attn_ws_bytes(queries->n_tokens, n_heads, d_v, k);
+  if (need && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
+    return DSA_ERR_WORKSPACE;
+  AttnLaunch L{cache, queries, q, n_heads, d_v, scale, idx, k, out, lse, workspace,
+               static_cast<cudaStream_t>(stream)};
+  return cuda_status(launch_attn(L));
+}
+
+dsa_status dsa_forward(const dsa_paged_cache* cache, const dsa_queries* queries,
+                       const uint8_t* q8, const float* q_scale, const float* w,
+                       int32_t n_idx_heads, const uint16_t* q, int32_t n_heads, int32_t d_v,
+                       float scale, int32_t k, uint16_t* out, float* lse, int32_t* idx_out,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status s = check_cache(cache, true, true);
+  if (s != DSA_OK) return s;
+  if ((s = check_queries(queries)) != DSA_OK) return s;
+  if (n_idx_heads < 1 || n_idx_heads > 64) return DSA_ERR_UNSUPPORTED;
+  if ((s = check_attn_shape(n_heads, cache->d_kv, d_v, k)) != DSA_OK) return s;
+  if (!(scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  const int T = queries->n_tokens;
+  if (T == 0) return DSA_OK;
+  if (!q8 || !q_scale || !w || !q || !out) return DSA_ERR_INVALID_ARG;
+  if (!aligned(q8, 16) || !aligned(q, 16) || !aligned(out, 16)) return DSA_ERR_INVALID_ARG;
+  const ForwardLayout FL = forward_layout(T, queries->max_pos, k, n_heads, d_v);
+  if (!workspace || workspace_bytes < FL.total || !aligned(workspace, 256))
+    return DSA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* logits = reinterpret_cast<float*>(ws + FL.logits);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + FL.idx);
+  IndexerLaunch IL{cache, queries, q8, q_scale, w, n_idx_heads, logits, FL.ld, ws + FL.plan, st};
+  if ((s = cuda_status(launch_indexer(IL))) != DSA_OK) return s;
+  if ((s = cuda_status(launch_topk(logits, FL.ld, queries, k, idx, nullptr, st))) != DSA_OK)
+    return s;
+  AttnLaunch AL{cache, queries, q, n_heads, d_v, scale, idx, k, out, lse, ws + FL.attn, st};
+  return cuda_status(launch_attn(AL));
+}
+
+dsa_status dsa_read_device_status(void* stream) {
+  uint32_t v = 0;
+  if (read_and_clear_status(static_cast<cudaStream_t>(stream), &v) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (v & kErrTimeout) return DSA_ERR_TIMEOUT;
+  if (v & kErrBadIndex) return DSA_ERR_BAD_INDEX;
+  return DSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,545 @@
+// Lightning indexer (DSA step 1) on sm_100a.
+//
+// I[t,s] = k_scale[s] * sum_j (w[t,j] * q_scale[t]) * ReLU(sum_d q8[t,j,d] * k8[s,d])
+// which equals sum_j w[t,j] * ReLU(qhat[t,j,:] . khat[s,:]) because both scales are
+// positive ("DeepSeek V3.2-Exp Cuts Prolonged-Context Costs ...", section "FP8 index ->
+// top-k selection -> sparse core attention", item (1): few FP8 heads with a ReLU, scoring
+// every preceding token).
+//
+// Design (B200): the FP8 products run on the 5th-gen tensor cores.  One MMA tile is
+// D[128 keys, N] = K8[128 keys, D_I] * Q8[N, D_I]^T with N = (tokens in the run) x (padded
+// heads), fp32 accumulators in TMEM, so each epilogue thread owns one key and has all of
+// its head values in registers: ReLU, the head weights and the causal mask are applied
+// without any cross-thread traffic.  Keys stream from the paged cache with TMA (one
+// 64-token page per box, swizzled for the MMA), through a multi-stage mbarrier ring.
+//
+//   warp 0      producer: Q rows of each run (manual swizzled stores) + TMA key pages
+//   warp 1      one thread issues tcgen05.mma (kind::f8f6f4) and tcgen05.commit
+//   warps 2..5  epilogue: tcgen05.ld -> ReLU . w -> logits (coalesced fp32 stores)
+//
+// A small planner kernel first groups the query tokens into runs of up to 4 tokens of
+// the same sequence (they share every key tile) and lays the (run, key tile) work items
+// out flat; the persistent CTAs then take equal contiguous slices of that list.
+#include <cudaTypedefs.h>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+// ---------------------------------------------------------------------------- plan
+// Workspace (int32 words): hdr[4] = {n_runs, total_items, -, -}, then per run:
+// tok0[T], ntok[T], seq[T], maxpos[T], and item0[T+1] (prefix sum of key tiles).
+struct PlanView {
+  int32_t* hdr;
+  int32_t* tok0;
+  int32_t* ntok;
+  int32_t* seq;
+  int32_t* maxpos;
+  int32_t* item0;
+};
+__host__ __device__ inline PlanView plan_view(void* ws, int32_t T) {
+  int32_t* p = static_cast<int32_t*>(ws);
+  PlanView v;
+  v.hdr = p;
+  p += 4;
+  v.tok0 = p;
+  p += T;
+  v.ntok = p;
+  p += T;
+  v.seq = p;
+  p += T;
+  v.maxpos = p;
+  p += T;
+  v.item0 = p;
+  return v;
+}
+
+size_t indexer_ws_bytes(int32_t T) {
+  const size_t words = 4 + 5 * static_cast<size_t>(T < 0 ? 0 : T) + 1;
+  return (words * 4 + 255) & ~static_cast<size_t>(255);
+}
+
+// Exclusive scan over a 1024-thread block.
+__device__ int block_excl_scan(int v, int* total, int* sm) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sm[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    const int t = (lane < static_cast<int>(blockDim.x >> 5)) ? sm[lane] : 0;
+    int tt = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, tt, o);
+      if (lane >= o) tt += y;
+    }
+    sm[lane] = tt - t;
+    if (lane == 31) sm[32] = tt;
+  }
+  __syncthreads();
+  const int res = sm[wid] + x - v;
+  *total = sm[32];
+  __syncthreads();
+  return res;
+}
+
+__global__ void __launch_bounds__(1024) indexer_plan_kernel(const int32_t* __restrict__ tok_seq,
+                                                            const int32_t* __restrict__ tok_pos,
+                                                            int32_t T, int32_t batch,
+                                                            int32_t max_pos, int32_t pos_cap,
+                                                            void* ws) {
+  __shared__ int sm[33];
+  PlanView v = plan_view(ws, T);
+  const int n_groups = (T + kRunTokens - 1) / kRunTokens;
+  int carry = 0;
+  for (int base = 0; base < n_groups; base += blockDim.x) {
+    const int g = base + threadIdx.x;
+    int nr = 0, cnt = 0, seqs[kRunTokens], poss[kRunTokens];
+    bool ok[kRunTokens], uniform = true;
+    if (g < n_groups) {
+      cnt = min(kRunTokens, T - kRunTokens * g);
+      for (int j = 0; j < cnt; ++j) {
+        const int t = kRunTokens * g + j;
+        seqs[j] = tok_seq[t];
+        poss[j] = tok_pos[t];
+        ok[j] = seqs[j] >= 0 && seqs[j] < batch && poss[j] >= 0 && poss[j] <= max_pos &&
+                poss[j] < pos_cap;
+        if (!ok[j]) {
+          record_error(kErrBadIndex);
+          uniform = false;
+        }
+        if (seqs[j] != seqs[0]) uniform = false;
+      }
+      nr = uniform ? 1 : cnt;
+    }
+    int total;
+    const int off = block_excl_scan(nr, &total, sm) + carry;
+    if (g < n_groups) {
+      if (uniform) {
+        int mp = poss[0];
+        for (int j = 1; j < cnt; ++j) mp = max(mp, poss[j]);
+        v.tok0[off] = kRunTokens * g;
+        v.ntok[off] = cnt;
+        v.seq[off] = seqs[0];
+        v.maxpos[off] = mp;
+      } else {
+        for (int j = 0; j < cnt; ++j) {
+          v.tok0[off + j] = kRunTokens * g + j;
+          v.ntok[off + j] = 1;
+          v.seq[off + j] = ok[j] ? seqs[j] : 0;
+          v.maxpos[off + j] = ok[j] ? poss[j] : -1;  // no work for an invalid token
+        }
+      }
+    }
+    carry += total;
+  }
+  const int n_runs = carry;
+  __syncthreads();
+  int icarry = 0;
+  for (int base = 0; base < n_runs; base += blockDim.x) {
+    const int r = base + threadIdx.x;
+    const int ni = r < n_runs ? (v.maxpos[r] + kKeyTile) / kKeyTile : 0;
+    int total;
+    const int off = block_excl_scan(ni, &total, sm) + icarry;
+    if (r < n_runs) v.item0[r] = off;
+    icarry += total;
+  }
+  if (threadIdx.x == 0) {
+    v.item0[n_runs] = icarry;
+    v.hdr[0] = n_runs;
+    v.hdr[1] = icarry;
+  }
+}
+
+// ---------------------------------------------------------------------------- main kernel
+struct IdxArgs {
+  const float* k_scale;
+  const int32_t* block_table;
+  int32_t max_blocks;
+  int32_t num_blocks;
+  const int32_t* tok_pos;
+  const uint8_t* q8;
+  const float* q_scale;
+  const float* w;
+  int32_t n_idx_heads;
+  float* logits;
+  int64_t ld;
+  void* plan;
+  int32_t T;
+};
+
+__host__ __device__ constexpr int pow2ceil(int x) {
+  int p = 32;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+template <int DI, int HP>
+struct IdxCfg {
+  static constexpr int kStages = DI == 128 ? 6 : 8;
+  static constexpr int kTileBytes = kKeyTile * DI;
+  static constexpr int kQBytes = kRunTokens * HP * DI;
+  static constexpr int kNC = kRunTokens * HP;  // TMEM columns of one accumulator buffer
+  static constexpr int kTmemCols = pow2ceil(2 * kNC);
+  static constexpr int kOffK = 0;
+  static constexpr int kOffQ = kOffK + kStages * kTileBytes;
+  static constexpr int kOffWq = kOffQ + 2 * kQBytes;
+  static constexpr int kOffMeta = kOffWq + 2 * kRunTokens * HP * 4;
+  static constexpr int kOffBar = kOffMeta + 64;
+  static constexpr int kNumBars = 2 * kStages + 9;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmem = kOffMisc + 16;
+  static constexpr int kSmemAlloc = kSmem + 1024;
+  static constexpr uint32_t kSwz = DI == 128 ? kSw128 : (DI == 64 ? kSw64 : kSw32);
+  static_assert(kTileBytes % 1024 == 0 && kQBytes % 1024 == 0, "tile alignment");
+};
+
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kWaitBudgetNs) return false;
+  }
+  return true;
+}
+
+// Walks this CTA's slice of the flat (run, tile) list in order; every role runs its
+// own copy so they agree on run boundaries without talking to each other.
+struct ItemWalker {
+  const int32_t* item0;
+  int i, i1, r, rc;
+  bool new_run, last_of_run;
+  int tile;
+  __device__ bool next() {
+    if (i >= i1) return false;
+    const int prev = r;
+    while (i >= item0[r + 1]) ++r;
+    new_run = (rc < 0) || (r != prev);
+    if (new_run) ++rc;
+    tile = i - item0[r];
+    last_of_run = (i + 1 >= i1) || (i + 1 >= item0[r + 1]);
+    return true;
+  }
+  __device__ void advance() { ++i; }
+};
+
+template <int DI, int HP>
+__global__ void __launch_bounds__(192, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap kmap, const IdxArgs a) {
+  using C = IdxCfg<DI, HP>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* ktiles = smem + C::kOffK;
+  uint8_t* qbuf = smem + C::kOffQ;
+  float* wq = reinterpret_cast<float*>(smem + C::kOffWq);
+  int* qpos = reinterpret_cast<int*>(smem + C::kOffMeta);
+  int* qtok = qpos + 2 * kRunTokens;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* qfull = bars + 2 * S;
+  uint64_t* qempty = qfull + 2;
+  uint64_t* tfull = qempty + 2;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  PlanView pv = plan_view(a.plan, a.T);
+  const int n_runs = pv.hdr[0];
+  const int total = pv.hdr[1];
+  const int i0 = static_cast<int>(static_cast<int64_t>(total) * blockIdx.x / gridDim.x);
+  const int i1 = static_cast<int>(static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x);
+  if (i0 >= i1) return;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&qfull[q], 1);
+      mbar_init(&qempty[q], 1 + 4);
+      mbar_init(&tfull[q], 1);
+      mbar_init(&tempty[q], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // run containing item i0
+  int lo = 0, hi = n_runs;  // item0[lo] <= i0 < item0[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (pv.item0[mid] <= i0) lo = mid;
+    else hi = mid;
+  }
+  ItemWalker wk{pv.item0, i0, i1, lo, -1, false, false, 0};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int n = 0;
+    for (; wk.next(); wk.advance(), ++n) {
+      const int r = wk.r;
+      if (wk.new_run) {
+        const int slot = wk.rc & 1;
+        if (!mbar_wait(&qempty[slot], ((wk.rc >> 1) & 1) ^ 1, abort_flag)) break;
+        const int tok0 = pv.tok0[r], ntok = pv.ntok[r];
+        uint8_t* qb = qbuf + slot * C::kQBytes;
+        constexpr int kChunks = DI / 16;
+        for (int c = lane; c < ntok * HP * kChunks; c += 32) {
+          const int row = c / kChunks, cc = c % kChunks;
+          const int j = row / HP, h = row % HP;
+          uint4 val = make_uint4(0, 0, 0, 0);
+          if (h < a.n_idx_heads)
+            val = *reinterpret_cast<const uint4*>(
+                a.q8 + (static_cast<size_t>(tok0 + j) * a.n_idx_heads + h) * DI + cc * 16);
+          *reinterpret_cast<uint4*>(qb + swz_offset(row, cc * 16, DI)) = val;
+        }
+        for (int e = lane; e < ntok * HP; e += 32) {
+          const int j = e / HP, h = e % HP;
+          wq[(slot * kRunTokens + j) * HP + h] =
+              h < a.n_idx_heads
+                  ? a.w[static_cast<size_t>(tok0 + j) * a.n_idx_heads + h] * a.q_scale[tok0 + j]
+                  : 0.f;
+        }
+        if (lane < ntok) {
+          qpos[slot * kRunTokens + lane] = a.tok_pos[tok0 + lane];
+          qtok[slot * kRunTokens + lane] = tok0 + lane;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qfull[slot]);
+      }
+      const int stage = n % S;
+      if (!mbar_wait(&empty[stage], ((n / S) & 1) ^ 1, abort_flag)) break;
+      if (lane == 0) {
+        const int seq = pv.seq[r], nblk = (pv.maxpos[r] + kPage) / kPage;
+        int pb[2];
+        uint32_t bytes = 0;
+        for (int h = 0; h < 2; ++h) {
+          const int lb = wk.tile * 2 + h;
+          pb[h] = -1;
+          if (lb < nblk) {
+            const int p = a.block_table[static_cast<size_t>(seq) * a.max_blocks + lb];
+            if (p >= 0 && p < a.num_blocks) pb[h] = p;
+            else record_error(kErrBadIndex);
+          }
+          if (pb[h] >= 0) bytes += kPage * DI;
+        }
+        if (bytes) mbar_arrive_expect_tx(&full[stage], bytes);
+        else mbar_arrive(&full[stage]);
+        for (int h = 0; h < 2; ++h)
+          if (pb[h] >= 0)
+            tma_load_2d(ktiles + stage * C::kTileBytes + h * kPage * DI, &kmap, &full[stage], 0,
+                        pb[h] * kPage);
+      }
+      __syncwarp();
+    }
+    // let every issued TMA land before the CTA can exit
+    if (lane == 0)
+      for (int m = max(0, n - S); m < n; ++m) mbar_wait_drain(&full[m % S], (m / S) & 1);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int n = 0;
+      int slot = 0;
+      for (; wk.next(); wk.advance(), ++n) {
+        const int r = wk.r;
+        if (wk.new_run) {
+          slot = wk.rc & 1;
+          if (!mbar_wait(&qfull[slot], (wk.rc >> 1) & 1, abort_flag)) break;
+        }
+        const int ab = n & 1;
+        if (!mbar_wait(&tempty[ab], ((n >> 1) & 1) ^ 1, abort_flag)) break;
+        const int stage = n % S;
+        if (!mbar_wait(&full[stage], (n / S) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t N = static_cast<uint32_t>(pv.ntok[r] * HP);
+        const uint32_t idesc = instr_desc(128, N, 0, 0, 0, 0);
+        const uint32_t a_base = smem_u32(ktiles + stage * C::kTileBytes);
+        const uint32_t b_base = smem_u32(qbuf + slot * C::kQBytes);
+#pragma unroll
+        for (int ks = 0; ks < DI / 32; ++ks)
+          mma_f8(tmem + ab * C::kNC, smem_desc(a_base + ks * 32, 16, 8 * DI, C::kSwz),
+                 smem_desc(b_base + ks * 32, 16, 8 * DI, C::kSwz), idesc, ks > 0 ? 1u : 0u);
+        mma_commit(&empty[stage]);
+        mma_commit(&tfull[ab]);
+        if (wk.last_of_run) mma_commit(&qempty[slot]);
+      }
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    int n = 0;
+    int slot = 0;
+    for (; wk.next(); wk.advance(), ++n) {
+      const int r = wk.r;
+      if (wk.new_run) {
+        slot = wk.rc & 1;
+        if (!mbar_wait(&qfull[slot], (wk.rc >> 1) & 1, abort_flag)) break;
+      }
+      const int ab = n & 1;
+      if (!mbar_wait(&tfull[ab], (n >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      const int s = wk.tile * kKeyTile + row;
+      const int ntok = pv.ntok[r];
+      float ks = __int_as_float(0x7fc00000);
+      if (s <= pv.maxpos[r]) {
+        const int p =
+            a.block_table[static_cast<size_t>(pv.seq[r]) * a.max_blocks + s / kPage];
+        if (p >= 0 && p < a.num_blocks) ks = a.k_scale[static_cast<size_t>(p) * kPage + s % kPage];
+      }
+      for (int j = 0; j < ntok; ++j) {
+        float x[HP];
+        const uint32_t taddr =
+            tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::kNC + j * HP;
+        if constexpr (HP % 32 == 0) {
+#pragma unroll
+          for (int c = 0; c < HP / 32; ++c) tmem_ld32(taddr + c * 32, x + c * 32);
+        } else {
+          tmem_ld16(taddr, x);
+        }
+        tmem_wait_ld();
+        if (s <= qpos[slot * kRunTokens + j]) {
+          const float* wv = wq + (slot * kRunTokens + j) * HP;
+          float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+          for (int h = 0; h < HP; h += 2) {
+            acc0 = fmaf(fmaxf(x[h], 0.f), wv[h], acc0);
+            acc1 = fmaf(fmaxf(x[h + 1], 0.f), wv[h + 1], acc1);
+          }
+          a.logits[static_cast<int64_t>(qtok[slot * kRunTokens + j]) * a.ld + s] =
+              (acc0 + acc1) * ks;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&tempty[ab]);
+        if (wk.last_of_run) mbar_arrive(&qempty[slot]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------- host
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+template <int DI, int HP>
+static cudaError_t launch_indexer_t(const IndexerLaunch& L, const CUtensorMap& map, int grid) {
+  using C = IdxCfg<DI, HP>;
+  static bool attr_set = false;  // per process; the attribute is per function, all devices
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(indexer_kernel<DI, HP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  IdxArgs a;
+  a.k_scale = L.cache->k_scale;
+  a.block_table = L.cache->block_table;
+  a.max_blocks = L.cache->max_blocks_per_seq;
+  a.num_blocks = L.cache->num_blocks;
+  a.tok_pos = L.queries->tok_pos;
+  a.q8 = L.q8;
+  a.q_scale = L.q_scale;
+  a.w = L.w;
+  a.n_idx_heads = L.n_idx_heads;
+  a.logits = L.logits;
+  a.ld = L.ld_logits;
+  a.plan = L.ws;
+  a.T = L.queries->n_tokens;
+  indexer_kernel<DI, HP><<<grid, 192, C::kSmemAlloc, L.stream>>>(map, a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_indexer(const IndexerLaunch& L) {
+  const dsa_paged_cache* c = L.cache;
+  const dsa_queries* q = L.queries;
+  const int T = q->n_tokens;
+  if (T == 0) return cudaSuccess;
+  indexer_plan_kernel<<<1, 1024, 0, L.stream>>>(q->tok_seq, q->tok_pos, T, c->batch, q->max_pos,
+                                                c->max_blocks_per_seq * kPage, L.ws);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  const int DI = c->idx_dim;
+  CUtensorMap map;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(DI),
+                        static_cast<cuuint64_t>(c->num_blocks) * kPage};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(DI)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(DI), static_cast<cuuint32_t>(kPage)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz = DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : DI == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                            : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(c->k8), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+
+  const int64_t tiles_ub = static_cast<int64_t>(T) * ((q->max_pos + kKeyTile) / kKeyTile);
+  const int grid = static_cast<int>(tiles_ub < num_sms() ? tiles_ub : num_sms());
+  if (grid <= 0) return cudaSuccess;
+  const int HP = L.n_idx_heads <= 16 ? 16 : (L.n_idx_heads <= 32 ? 32 : 64);
+#define DSA_IDX_CASE(di, hp) \
+  if (DI == di && HP == hp) return launch_indexer_t<di, hp>(L, map, grid);
+  DSA_IDX_CASE(128, 64)
+  DSA_IDX_CASE(128, 32)
+  DSA_IDX_CASE(128, 16)
+  DSA_IDX_CASE(64, 64)
+  DSA_IDX_CASE(64, 32)
+  DSA_IDX_CASE(64, 16)
+  DSA_IDX_CASE(32, 64)
+  DSA_IDX_CASE(32, 32)
+  DSA_IDX_CASE(32, 16)
+#undef DSA_IDX_CASE
+  return cudaErrorNotSupported;
+}
+
+}  // namespace dsa

@@ -1,0 +1,290 @@
+// Fine-grained token selection (DSA step 2): the k largest index logits of each query row.
+//
+// "DeepSeek V3.2-Exp Cuts Prolonged-Context Costs ...", section "FP8 index -> top-k
+// selection -> sparse core attention", item (2): keep only the top-k (k = 2048) key
+// entries per query.  Equal logits: the smaller position wins; fewer than k valid
+// positions: all of them are selected.
+//
+// Radix select, no sort.  A logit becomes an order-preserving uint32 key (sign bit
+// flipped for positives, all bits inverted for negatives).  Digits of 11, 11 and 10 bits
+// are resolved from the top with shared-memory histograms (warp-aggregated atomics via
+// __match_any_sync) and a block-wide suffix scan.  After the first digit every element of
+// a higher bucket is already selected and is written out at once; the elements of the
+// threshold bucket are gathered (in position order) into a shared candidate list, and
+// the two remaining digits run on that list only.  All writes are ordered compactions
+// (warp ballots + a block scan), so the result is deterministic.
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+constexpr int kTopkThreads = 1024;
+constexpr int kTopkCand = 8192;       // threshold-bucket candidates kept in shared memory
+constexpr int kTopkRowCache = 32768;  // rows up to this length are cached in shared memory
+
+struct TopkSmem {
+  uint32_t hist[2048];
+  int scan[72];
+  int sel[4];
+  uint32_t cand_key[kTopkCand];
+  int32_t cand_idx[kTopkCand];
+};
+constexpr size_t kTopkSmemBase = sizeof(TopkSmem);
+constexpr size_t kTopkSmemMax = kTopkSmemBase + kTopkRowCache * sizeof(uint32_t);
+
+size_t topk_ws_bytes(int32_t, int32_t, int32_t) { return 0; }
+
+struct RowGlobal {
+  const float* row;
+  __device__ uint32_t key(int i) const { return float_to_ordered(row[i]); }
+  __device__ int index(int i) const { return i; }
+};
+struct RowCached {
+  const uint32_t* keys;
+  __device__ uint32_t key(int i) const { return keys[i]; }
+  __device__ int index(int i) const { return i; }
+};
+struct RowCand {
+  const uint32_t* keys;
+  const int32_t* idx;
+  __device__ uint32_t key(int i) const { return keys[i]; }
+  __device__ int index(int i) const { return idx[i]; }
+};
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Block-wide exclusive scan of two counters per warp (warp totals in sm->scan).
+// Returns per-warp exclusive offsets for class A and class B and the block totals.
+__device__ __forceinline__ void scan_two(TopkSmem* sm, int wa, int wb, int* off_a, int* off_b,
+                                         int* tot_a, int* tot_b) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0) {
+    sm->scan[wid] = wa;
+    sm->scan[32 + wid] = wb;
+  }
+  __syncthreads();
+  if (wid == 0) {
+    int a = sm->scan[lane], b = sm->scan[32 + lane];
+    int ia = a, ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, ia, o), yb = __shfl_up_sync(0xffffffffu, ib, o);
+      if (lane >= o) {
+        ia += ya;
+        ib += yb;
+      }
+    }
+    sm->scan[lane] = ia - a;
+    sm->scan[32 + lane] = ib - b;
+    if (lane == 31) {
+      sm->scan[64] = ia;
+      sm->scan[65] = ib;
+    }
+  }
+  __syncthreads();
+  *off_a = sm->scan[wid];
+  *off_b = sm->scan[32 + wid];
+  *tot_a = sm->scan[64];
+  *tot_b = sm->scan[65];
+  __syncthreads();
+}
+
+// Histogram of digit = (key >> shift) & (nb-1) over elements with (key >> pshift) == prefix
+// (pshift == 32: every element).
+template <class Src>
+__device__ void hist_pass(TopkSmem* sm, const Src& src, int n, int shift, int nb, int pshift,
+                          uint32_t prefix) {
+  for (int b = threadIdx.x; b < 2048; b += blockDim.x) sm->hist[b] = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    bool take = false;
+    uint32_t d = 0;
+    if (i < n) {
+      const uint32_t k = src.key(i);
+      take = pshift >= 32 || (k >> pshift) == prefix;
+      d = (k >> shift) & static_cast<uint32_t>(nb - 1);
+    }
+    const uint32_t active = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const uint32_t peers = __match_any_sync(active, d);
+      if ((lanemask_lt() & peers) == 0) atomicAdd(&sm->hist[d], __popc(peers));
+    }
+  }
+  __syncthreads();
+}
+
+// Largest bucket b with count(> b) < k_rem <= count(>= b).  Writes sel[0] = b,
+// sel[1] = count(> b).
+__device__ void select_bucket(TopkSmem* sm, int nb, int k_rem) {
+  const int t = threadIdx.x;
+  const int b0 = nb - 1 - 2 * t, b1 = b0 - 1;
+  const int c0 = b0 >= 0 ? static_cast<int>(sm->hist[b0]) : 0;
+  const int c1 = b1 >= 0 ? static_cast<int>(sm->hist[b1]) : 0;
+  // inclusive scan of (c0 + c1) in descending bucket order
+  const int lane = t & 31, wid = t >> 5;
+  int x = c0 + c1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sm->scan[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    const int v = sm->scan[lane];
+    int iv = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, iv, o);
+      if (lane >= o) iv += y;
+    }
+    sm->scan[lane] = iv - v;
+  }
+  __syncthreads();
+  const int excl = sm->scan[wid] + x - (c0 + c1);
+  if (b0 >= 0 && excl < k_rem && excl + c0 >= k_rem) {
+    sm->sel[0] = b0;
+    sm->sel[1] = excl;
+  }
+  if (b1 >= 0 && excl + c0 < k_rem && excl + c0 + c1 >= k_rem) {
+    sm->sel[0] = b1;
+    sm->sel[1] = excl + c0;
+    sm->sel[2] = c1;
+  }
+  if (b0 >= 0 && excl < k_rem && excl + c0 >= k_rem) sm->sel[2] = c0;
+  __syncthreads();
+}
+
+// One ordered pass: class A elements go to outA[baseA + rank]; class B elements with
+// rank < limitB go to the B sink.  cls(key) -> 0 none, 1 A, 2 B.
+template <class Src, class Cls, class SinkB>
+__device__ void ordered_pass(TopkSmem* sm, const Src& src, int n, Cls cls, int32_t* outA,
+                             int baseA, SinkB sinkB, int limitB) {
+  const int lane = threadIdx.x & 31;
+  int run_a = 0, run_b = 0;
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    int c = 0;
+    uint32_t key = 0;
+    if (i < n) {
+      key = src.key(i);
+      c = cls(key);
+    }
+    const uint32_t ba = __ballot_sync(0xffffffffu, c == 1);
+    const uint32_t bb = __ballot_sync(0xffffffffu, c == 2);
+    int off_a, off_b, tot_a, tot_b;
+    scan_two(sm, __popc(ba), __popc(bb), &off_a, &off_b, &tot_a, &tot_b);
+    if (c == 1) outA[baseA + run_a + off_a + __popc(ba & lanemask_lt())] = src.index(i);
+    if (c == 2) {
+      const int rb = run_b + off_b + __popc(bb & lanemask_lt());
+      if (rb < limitB) sinkB(rb, key, src.index(i));
+    }
+    run_a += tot_a;
+    run_b += tot_b;
+  }
+}
+
+template <class Src>
+__device__ void select_from(TopkSmem* sm, const Src& src, int n, int k, int32_t* out) {
+  // digit 1: bits 21..31
+  hist_pass(sm, src, n, 21, 2048, 32, 0u);
+  select_bucket(sm, 2048, k);
+  const uint32_t b1 = static_cast<uint32_t>(sm->sel[0]);
+  const int above1 = sm->sel[1];
+  const int n_cand = sm->sel[2];
+  const int k2 = k - above1;
+  if (n_cand <= kTopkCand) {
+    // higher buckets are final; gather the threshold bucket in position order
+    ordered_pass(
+        sm, src, n, [b1](uint32_t key) { return (key >> 21) > b1 ? 1 : ((key >> 21) == b1 ? 2 : 0); },
+        out, 0,
+        [sm](int r, uint32_t key, int idx) {
+          sm->cand_key[r] = key;
+          sm->cand_idx[r] = idx;
+        },
+        kTopkCand);
+    __syncthreads();
+    RowCand cs{sm->cand_key, sm->cand_idx};
+    hist_pass(sm, cs, n_cand, 10, 2048, 32, 0u);
+    select_bucket(sm, 2048, k2);
+    const uint32_t b2 = static_cast<uint32_t>(sm->sel[0]);
+    const int above2 = sm->sel[1];
+    hist_pass(sm, cs, n_cand, 0, 1024, 10, (b1 << 11) | b2);
+    select_bucket(sm, 1024, k2 - above2);
+    const uint32_t thr = (b1 << 21) | (b2 << 10) | static_cast<uint32_t>(sm->sel[0]);
+    const int need_eq = k2 - above2 - sm->sel[1];
+    int32_t* eq_out = out + above1 + (k2 - need_eq);
+    ordered_pass(
+        sm, cs, n_cand, [thr](uint32_t key) { return key > thr ? 1 : (key == thr ? 2 : 0); },
+        out, above1, [eq_out](int r, uint32_t, int idx) { eq_out[r] = idx; }, need_eq);
+  } else {
+    hist_pass(sm, src, n, 10, 2048, 21, b1);
+    select_bucket(sm, 2048, k2);
+    const uint32_t b2 = static_cast<uint32_t>(sm->sel[0]);
+    const int above2 = sm->sel[1];
+    hist_pass(sm, src, n, 0, 1024, 10, (b1 << 11) | b2);
+    select_bucket(sm, 1024, k2 - above2);
+    const uint32_t thr = (b1 << 21) | (b2 << 10) | static_cast<uint32_t>(sm->sel[0]);
+    const int need_eq = k2 - above2 - sm->sel[1];
+    int32_t* eq_out = out + (k - need_eq);
+    ordered_pass(
+        sm, src, n, [thr](uint32_t key) { return key > thr ? 1 : (key == thr ? 2 : 0); }, out, 0,
+        [eq_out](int r, uint32_t, int idx) { eq_out[r] = idx; }, need_eq);
+  }
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1)
+    topk_kernel(const float* __restrict__ logits, int64_t ld, const int32_t* __restrict__ tok_pos,
+                int32_t max_pos, int32_t k, int32_t* __restrict__ idx, int cache_ok) {
+  extern __shared__ uint8_t topk_smem_raw[];
+  TopkSmem* sm = reinterpret_cast<TopkSmem*>(topk_smem_raw);
+  uint32_t* row_cache = reinterpret_cast<uint32_t*>(topk_smem_raw + kTopkSmemBase);
+  const int t = blockIdx.x;
+  int32_t* out = idx + static_cast<int64_t>(t) * k;
+  const int pos = tok_pos[t];
+  if (pos < 0 || pos > max_pos) {
+    if (threadIdx.x == 0) record_error(kErrBadIndex);
+    for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
+    return;
+  }
+  const int n = pos + 1;
+  const float* row = logits + static_cast<int64_t>(t) * ld;
+  if (n <= k) {
+    for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = i < n ? i : -1;
+    return;
+  }
+  if (cache_ok && n <= kTopkRowCache) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) row_cache[i] = float_to_ordered(row[i]);
+    __syncthreads();
+    select_from(sm, RowCached{row_cache}, n, k, out);
+  } else {
+    select_from(sm, RowGlobal{row}, n, k, out);
+  }
+}
+
+cudaError_t launch_topk(const float* logits, int64_t ld, const dsa_queries* q, int32_t k,
+                        int32_t* idx, void*, cudaStream_t stream) {
+  if (q->n_tokens == 0) return cudaSuccess;
+  const int cache_ok = (q->max_pos + 1) <= kTopkRowCache ? 1 : 0;
+  const size_t smem = cache_ok ? kTopkSmemMax : kTopkSmemBase;
+  static int attr_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kTopkSmemMax));
+    if (e != cudaSuccess) return e;
+    attr_dev = dev;
+  }
+  topk_kernel<<<q->n_tokens, kTopkThreads, smem, stream>>>(logits, ld, q->tok_pos, q->max_pos, k,
+                                                           idx, cache_ok);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -1,0 +1,206 @@
+"""Thin Python binding of libdsa.so (ctypes; argument marshalling only).
+
+Each function takes torch CUDA tensors, passes their device pointers and the current
+torch stream to the C entry point of the same name (include/dsa.h) and raises
+``DsaError`` on a non-OK status.  Every step of the computation runs in the library's
+sm_100a kernels; if the library cannot be loaded, the calls raise — there is no CPU
+fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+_LIB = None
+
+DSA_OK = 0
+STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
+                3: "DSA_ERR_WORKSPACE", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_BAD_INDEX",
+                6: "DSA_ERR_TIMEOUT"}
+
+EXPORTED = ("dsa_indexer_logits", "dsa_indexer_workspace_size", "dsa_topk",
+            "dsa_topk_workspace_size", "dsa_sparse_mla_attn", "dsa_attn_workspace_size",
+            "dsa_forward", "dsa_forward_workspace_size", "dsa_read_device_status",
+            "dsa_launch_count", "dsa_status_string", "dsa_abi_version")
+
+
+class DsaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} -> {STATUS_NAMES.get(status, status)}: "
+                         f"{lib().dsa_status_string(status).decode()}")
+
+
+class PagedCache(ctypes.Structure):
+    _fields_ = [("k8", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("kv", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("batch", ctypes.c_int32),
+                ("max_blocks_per_seq", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("idx_dim", ctypes.c_int32),
+                ("d_kv", ctypes.c_int32)]
+
+
+class Queries(ctypes.Structure):
+    _fields_ = [("n_tokens", ctypes.c_int32), ("tok_seq", ctypes.c_void_p),
+                ("tok_pos", ctypes.c_void_p), ("max_pos", ctypes.c_int32)]
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdsa.so (building it first if the sources are newer)."""
+    global _LIB
+    if _LIB is None:
+        path = lib_path()
+        if not _build.up_to_date():
+            try:
+                _build.build()
+            except Exception:
+                if not os.path.exists(path):
+                    raise
+        if not os.path.exists(path):
+            raise RuntimeError(f"libdsa.so not found at {path}; run the package build")
+        L = ctypes.CDLL(path)
+        P, I32, I64, SZ, F32 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t,
+                                ctypes.c_float)
+        PC, PQ = ctypes.POINTER(PagedCache), ctypes.POINTER(Queries)
+        sig = {
+            "dsa_indexer_logits": (I32, [PC, PQ, P, P, P, I32, P, I64, P, SZ, P]),
+            "dsa_indexer_workspace_size": (SZ, [I32]),
+            "dsa_topk": (I32, [P, I64, PQ, I32, P, P, SZ, P]),
+            "dsa_topk_workspace_size": (SZ, [I32, I32, I32]),
+            "dsa_sparse_mla_attn": (I32, [PC, PQ, P, I32, I32, F32, P, I32, P, P, P, SZ, P]),
+            "dsa_attn_workspace_size": (SZ, [I32, I32, I32, I32]),
+            "dsa_forward": (I32, [PC, PQ, P, P, P, I32, P, I32, I32, F32, I32, P, P, P, P, SZ, P]),
+            "dsa_forward_workspace_size": (SZ, [I32, I32, I32, I32, I32]),
+            "dsa_read_device_status": (I32, [P]),
+            "dsa_launch_count": (I64, []),
+            "dsa_status_string": (ctypes.c_char_p, [I32]),
+            "dsa_abi_version": (I32, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _LIB = L
+    return _LIB
+
+
+# ------------------------------------------------------------------------------ helpers
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libdsa takes CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("libdsa takes contiguous tensors only")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != DSA_OK:
+        raise DsaError(fn, status)
+
+
+def make_cache(k8: torch.Tensor, k_scale: torch.Tensor, kv: Optional[torch.Tensor],
+               block_table: torch.Tensor, page_size: int = 64) -> PagedCache:
+    """Describe device caches: k8 uint8 [rows, D_I], k_scale fp32 [rows],
+    kv uint16/int16/bf16 [rows, D_kv], block_table int32 [B, max_blocks]."""
+    rows = k8.shape[0] if k8 is not None else kv.shape[0]
+    return PagedCache(
+        _ptr(k8), _ptr(k_scale), _ptr(kv), _ptr(block_table), block_table.shape[0],
+        block_table.shape[1], rows // page_size, page_size,
+        k8.shape[1] if k8 is not None else 0, kv.shape[1] if kv is not None else 0)
+
+
+def make_queries(tok_seq: torch.Tensor, tok_pos: torch.Tensor, max_pos: int) -> Queries:
+    return Queries(tok_seq.shape[0], _ptr(tok_seq), _ptr(tok_pos), int(max_pos))
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------------------ entry points
+
+def dsa_indexer_logits(cache: PagedCache, queries: Queries, q8, q_scale, w, logits,
+                       workspace=None, stream=None):
+    """(1) logits[t, s] = sum_j w[t,j] ReLU(qhat[t,j] . khat[s]) for s <= tok_pos[t]."""
+    T = queries.n_tokens
+    need = lib().dsa_indexer_workspace_size(T)
+    if workspace is None:
+        workspace = _workspace(need, logits.device)
+    st = lib().dsa_indexer_logits(ctypes.byref(cache), ctypes.byref(queries), _ptr(q8),
+                                  _ptr(q_scale), _ptr(w), q8.shape[1], _ptr(logits),
+                                  logits.shape[1], _ptr(workspace), workspace.numel(),
+                                  _stream(stream))
+    _check("dsa_indexer_logits", st)
+    return logits
+
+
+def dsa_topk(logits, queries: Queries, k: int, idx, workspace=None, stream=None):
+    """(2) idx[t, :] = the positions of the k largest logits of row t (-1 padded)."""
+    need = lib().dsa_topk_workspace_size(queries.n_tokens, queries.max_pos, k)
+    if workspace is None and need:
+        workspace = _workspace(need, logits.device)
+    st = lib().dsa_topk(_ptr(logits), logits.shape[1], ctypes.byref(queries), k, _ptr(idx),
+                        _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                        _stream(stream))
+    _check("dsa_topk", st)
+    return idx
+
+
+def dsa_sparse_mla_attn(cache: PagedCache, queries: Queries, q, d_v: int, scale: float, idx,
+                        out, lse=None, workspace=None, stream=None):
+    """(3) out[t,h] = softmax over the selected latent rows of scale*q.kv, times kv[:, :d_v]."""
+    T, H = q.shape[0], q.shape[1]
+    k = idx.shape[1]
+    need = lib().dsa_attn_workspace_size(T, H, d_v, k)
+    if workspace is None and need:
+        workspace = _workspace(need, q.device)
+    st = lib().dsa_sparse_mla_attn(ctypes.byref(cache), ctypes.byref(queries), _ptr(q), H, d_v,
+                                   float(scale), _ptr(idx), k, _ptr(out), _ptr(lse),
+                                   _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                   _stream(stream))
+    _check("dsa_sparse_mla_attn", st)
+    return out
+
+
+def forward_workspace_size(n_tokens: int, max_pos: int, k: int, n_heads: int, d_v: int) -> int:
+    return int(lib().dsa_forward_workspace_size(n_tokens, max_pos, k, n_heads, d_v))
+
+
+def dsa_forward(cache: PagedCache, queries: Queries, q8, q_scale, w, q, d_v: int, scale: float,
+                k: int, out, lse=None, idx_out=None, workspace=None, stream=None):
+    """(1) + (2) + (3) in one call."""
+    T, H = q.shape[0], q.shape[1]
+    need = forward_workspace_size(T, queries.max_pos, k, H, d_v)
+    if workspace is None:
+        workspace = _workspace(need, q.device)
+    st = lib().dsa_forward(ctypes.byref(cache), ctypes.byref(queries), _ptr(q8), _ptr(q_scale),
+                           _ptr(w), q8.shape[1], _ptr(q), H, d_v, float(scale), k, _ptr(out),
+                           _ptr(lse), _ptr(idx_out), _ptr(workspace), workspace.numel(),
+                           _stream(stream))
+    _check("dsa_forward", st)
+    return out
+
+
+def dsa_read_device_status(stream=None) -> int:
+    """Waits for the stream; returns and clears the device status word (0 = OK)."""
+    return int(lib().dsa_read_device_status(_stream(stream)))
+
+
+def dsa_launch_count() -> int:
+    return int(lib().dsa_launch_count())

@@ -1,0 +1,100 @@
+"""The C ABI: libdsa.so builds for sm_100a, loads, exports every entry point that
+include/dsa.h declares, and rejects bad arguments on the host (no GPU needed: these
+checks return before any CUDA call)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_long_03_b200 import build, dsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    return sorted(set(re.findall(r"DSA_API[^;{]*?\b(dsa_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for required in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward"):
+        assert required in names
+    assert set(names) == set(dsa.EXPORTED)
+
+
+def test_library_builds_and_exports_every_symbol():
+    path = build.build()
+    assert os.path.exists(path)
+    L = ctypes.CDLL(path)
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    assert dsa.lib().dsa_abi_version() == 1
+    assert dsa.lib().dsa_status_string(3) == b"workspace too small"
+
+
+def _cache(**kw):
+    c = dict(k8=16, k_scale=16, kv=16, block_table=16, batch=1, max_blocks_per_seq=8,
+             num_blocks=8, page_size=64, idx_dim=128, d_kv=576)
+    c.update(kw)
+    return dsa.PagedCache(**c)
+
+
+def _q(**kw):
+    q = dict(n_tokens=4, tok_seq=16, tok_pos=16, max_pos=511)
+    q.update(kw)
+    return dsa.Queries(**q)
+
+
+def _indexer(cache, queries, n_idx_heads=64, ld=512, ws=256, ws_bytes=1 << 20):
+    L = dsa.lib()
+    return L.dsa_indexer_logits(ctypes.byref(cache), ctypes.byref(queries), 16, 16, 16,
+                                n_idx_heads, 16, ld, ws, ws_bytes, None)
+
+
+def test_indexer_validation():
+    assert _indexer(_cache(page_size=32), _q()) == 2
+    assert _indexer(_cache(idx_dim=96), _q()) == 2
+    assert _indexer(_cache(), _q(), n_idx_heads=65) == 2
+    assert _indexer(_cache(block_table=None), _q()) == 1
+    assert _indexer(_cache(), _q(), ld=100) == 1
+    assert _indexer(_cache(), _q(max_pos=-1)) == 1
+    assert _indexer(_cache(k8=17), _q()) == 1  # misaligned
+    assert _indexer(_cache(), _q(), ws_bytes=8) == 3
+    assert _indexer(_cache(), _q(), ws=None) == 3
+    assert _indexer(_cache(), _q(n_tokens=0)) == 0  # nothing to do, nothing launched
+
+
+def test_topk_validation():
+    L = dsa.lib()
+    q = _q()
+    assert L.dsa_topk(16, 512, ctypes.byref(q), 0, 16, None, 0, None) == 2
+    assert L.dsa_topk(16, 512, ctypes.byref(q), 4096, 16, None, 0, None) == 2
+    assert L.dsa_topk(None, 512, ctypes.byref(q), 2048, 16, None, 0, None) == 1
+    assert L.dsa_topk(16, 10, ctypes.byref(q), 2048, 16, None, 0, None) == 1
+
+
+def _attn(cache, queries, H=128, d_v=512, scale=0.07, k=2048, q=16, out=16):
+    L = dsa.lib()
+    return L.dsa_sparse_mla_attn(ctypes.byref(cache), ctypes.byref(queries), q, H, d_v, scale,
+                                 16, k, out, None, 256, 1 << 30, None)
+
+
+def test_attention_validation():
+    assert _attn(_cache(), _q(), H=129) == 2
+    assert _attn(_cache(), _q(), d_v=500) == 2
+    assert _attn(_cache(d_kv=600), _q()) == 2
+    assert _attn(_cache(d_kv=40), _q(), d_v=64) == 2  # d_v > d_kv
+    assert _attn(_cache(), _q(), k=0) == 2
+    assert _attn(_cache(), _q(), scale=-1.0) == 1
+    assert _attn(_cache(), _q(), q=None) == 1
+    assert _attn(_cache(kv=None), _q()) == 1
+
+
+def test_forward_workspace_size_grows_with_context():
+    a = dsa.forward_workspace_size(4, 65535, 2048, 128, 512)
+    b = dsa.forward_workspace_size(4, 131071, 2048, 128, 512)
+    assert b > a > 4 * 65536 * 4
+    assert dsa.forward_workspace_size(0, 0, 2048, 128, 512) >= 0
