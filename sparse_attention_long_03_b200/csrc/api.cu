@@ -86,9 +86,13 @@ static dsa_status check_attn_shape(int32_t n_heads, int32_t d_kv, int32_t d_v, i
 }
 
 // Forward workspace: [indexer plan][logits T x ld][idx T x k][attention partials]
+// [decode top-k region: histogram, counters, scratch] (the last only for few rows)
+constexpr int kDecodeMaxRows = 64;
 struct ForwardLayout {
-  size_t plan, logits, idx, attn, total;
+  size_t plan, logits, idx, attn, topk, total;
   int64_t ld;
+  bool decode;
+  int chunks;
 };
 static ForwardLayout forward_layout(int32_t T, int32_t max_pos, int32_t k, int32_t H,
                                     int32_t d_v) {
@@ -102,6 +106,10 @@ static ForwardLayout forward_layout(int32_t T, int32_t max_pos, int32_t k, int32
   off += align256(static_cast<size_t>(T) * k * 4);
   L.attn = off;
   off += align256(attn_ws_bytes(T, H, d_v, k));
+  L.topk = off;
+  L.decode = T <= kDecodeMaxRows;
+  L.chunks = L.decode ? topk_decode_chunks(T, max_pos) : 0;
+  if (L.decode) off += align256(topk_decode_ws_bytes(T, L.ld, L.chunks));
   L.total = off;
   return L;
 }
@@ -222,9 +230,22 @@ dsa_status dsa_forward(const dsa_paged_cache* cache, const dsa_queries* queries,
   float* logits = reinterpret_cast<float*>(ws + FL.logits);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + FL.idx);
   IndexerLaunch IL{cache, queries, q8, q_scale, w, n_idx_heads, logits, FL.ld, ws + FL.plan, st};
-  if ((s = cuda_status(launch_indexer(IL))) != DSA_OK) return s;
-  if ((s = cuda_status(launch_topk(logits, FL.ld, queries, k, idx, nullptr, st))) != DSA_OK)
-    return s;
+  if (FL.decode) {
+    // few long rows: the indexer also builds the first-digit histogram and the top-k
+    // spreads each row over several CTAs
+    const TopkDecodeLayout TL = topk_decode_layout(ws + FL.topk, T, FL.ld, FL.chunks);
+    IL.hist = TL.hist;
+    IL.zero = TL.hist;
+    IL.zero_words = TL.zero_words;
+    if ((s = cuda_status(launch_indexer(IL))) != DSA_OK) return s;
+    if ((s = cuda_status(launch_topk_decode(logits, FL.ld, queries, k, idx, TL, FL.chunks, st))) !=
+        DSA_OK)
+      return s;
+  } else {
+    if ((s = cuda_status(launch_indexer(IL))) != DSA_OK) return s;
+    if ((s = cuda_status(launch_topk(logits, FL.ld, queries, k, idx, nullptr, st))) != DSA_OK)
+      return s;
+  }
   AttnLaunch AL{cache, queries, q, n_heads, d_v, scale, idx, k, out, lse, ws + FL.attn, st};
   return cuda_status(launch_attn(AL));
 }

@@ -198,6 +198,7 @@ __global__ void __launch_bounds__(192, 1) __cluster_dims__(2, 1, 1)
   __syncthreads();
   cluster_sync();  // the peer's barriers are initialised before anyone arrives remotely
   tc_fence_after();
+  pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tmem_o = tmem + 2 * kBN;
 
@@ -217,6 +218,7 @@ __global__ void __launch_bounds__(192, 1) __cluster_dims__(2, 1, 1)
       cp_async_16(qs + oc * kQChunk + swz_offset(h, c16 * 16, 128), src, valid * 2);
     }
     cp_async_arrive_noinc(q_full);
+    pdl_wait();  // the selection comes from the previous kernel
     int i = 0;
     for (; i < n_tiles; ++i) {
       const int st = i & 1;
@@ -244,6 +246,7 @@ __global__ void __launch_bounds__(192, 1) __cluster_dims__(2, 1, 1)
     cp_async_wait<0>();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    pdl_wait();
     if (lane == 0) {
       const uint32_t idesc_s = instr_desc(128, kBN, 1, 1, 0, 0);
       const uint32_t idesc_pv = instr_desc(128, cp.nvo > 0 ? cp.nvo * 64 : 64, 1, 1, 0, 1);
@@ -299,6 +302,7 @@ __global__ void __launch_bounds__(192, 1) __cluster_dims__(2, 1, 1)
     const int h = quarter * 32 + lane;  // head row == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t x_peer = map_peer(smem_u32(xs + h * kBN), peer);
+    pdl_wait();
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
@@ -483,6 +487,8 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restri
   const int t = blockIdx.y, h = blockIdx.x;
   __shared__ float wsh[64];
   __shared__ float lse_sh;
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x < 32) {
     float m = -INFINITY;
     for (int s = threadIdx.x; s < splits; s += 32)
@@ -584,15 +590,11 @@ cudaError_t launch_attn(const AttnLaunch& L) {
     a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(L.ws) +
                                           ((o + 255) & ~static_cast<size_t>(255)));
   }
-  dim3 grid(2 * splits, T);
-  sparse_mla_kernel<<<grid, 192, attn::kSmemAlloc, L.stream>>>(a);
-  count_launch();
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(sparse_mla_kernel, dim3(2 * splits, T), dim3(192), attn::kSmemAlloc,
+                             L.stream, a);
   if (e != cudaSuccess || splits == 1) return e;
-  attn_combine_kernel<<<dim3(L.n_heads, T), 128, 0, L.stream>>>(a.part_o, a.part_lse, splits,
-                                                                L.n_heads, L.d_v, L.out, L.lse);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(attn_combine_kernel, dim3(L.n_heads, T), dim3(128), 0, L.stream, a.part_o,
+                    a.part_lse, splits, L.n_heads, L.d_v, L.out, L.lse);
 }
 
 }  // namespace dsa

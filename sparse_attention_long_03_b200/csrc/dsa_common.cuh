@@ -273,6 +273,17 @@ __device__ __forceinline__ uint32_t swz_offset(uint32_t r, uint32_t c, uint32_t 
   return r * row_bytes + ((chunk ^ x) << 4) + (c & 15u);
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while the previous
+// kernel in the stream is still running.  pdl_wait() blocks until that kernel has
+// completed and its writes are visible: call it before touching anything the previous
+// kernel writes or reads.  pdl_trigger() lets the next kernel start its prologue early.
+// Both are no-ops when the kernel was launched normally.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ misc
 // Order-preserving uint32 image of a float (-0.0 is mapped like +0.0).
 __device__ __forceinline__ uint32_t float_to_ordered(float f) {

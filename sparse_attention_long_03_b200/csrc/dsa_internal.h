@@ -18,6 +18,26 @@ constexpr int kMaxTopK = 2048;
 void count_launch();
 int num_sms();
 
+// Launch `kernel` on `stream` with programmatic stream serialisation (the kernel may
+// overlap the tail of the previous kernel in the stream; it must call pdl_wait()).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  count_launch();
+  return e;
+}
+
 // ---- indexer ------------------------------------------------------------------------
 size_t indexer_ws_bytes(int32_t n_tokens);
 struct IndexerLaunch {
@@ -31,6 +51,9 @@ struct IndexerLaunch {
   int64_t ld_logits;
   void* ws;
   cudaStream_t stream;
+  uint32_t* hist = nullptr;     // optional [T][2048] first-digit histogram of the logits
+  uint32_t* zero = nullptr;     // region the prep kernel zeroes first (histogram, counters)
+  int64_t zero_words = 0;
 };
 cudaError_t launch_indexer(const IndexerLaunch& a);
 
@@ -38,6 +61,21 @@ cudaError_t launch_indexer(const IndexerLaunch& a);
 size_t topk_ws_bytes(int32_t n_tokens, int32_t max_pos, int32_t k);
 cudaError_t launch_topk(const float* logits, int64_t ld, const dsa_queries* q, int32_t k,
                         int32_t* idx, void* ws, cudaStream_t stream);
+// decode variant: several CTAs per row, first digit from the indexer's histogram
+struct TopkDecodeLayout {
+  uint32_t* hist;
+  uint32_t* arrive;
+  int64_t zero_words;  // hist + arrive, from the start of the region
+  int32_t* counts;
+  int32_t* scr_a;
+  int32_t* scr_b;
+};
+size_t topk_decode_ws_bytes(int32_t T, int64_t ld, int chunks);
+int topk_decode_chunks(int32_t T, int32_t max_pos);
+TopkDecodeLayout topk_decode_layout(void* ws, int32_t T, int64_t ld, int chunks);
+cudaError_t launch_topk_decode(const float* logits, int64_t ld, const dsa_queries* q, int32_t k,
+                               int32_t* idx, const TopkDecodeLayout& L, int chunks,
+                               cudaStream_t stream);
 
 // ---- sparse MLA attention --------------------------------------------------------------
 size_t attn_ws_bytes(int32_t n_tokens, int32_t n_heads, int32_t d_v, int32_t k);

@@ -89,12 +89,18 @@ __device__ int block_excl_scan(int v, int* total, int* sm) {
   return res;
 }
 
-__global__ void __launch_bounds__(1024) indexer_plan_kernel(const int32_t* __restrict__ tok_seq,
+// Plans the indexer work and zeroes `zero_words` words at `zero` (the top-k histogram and
+// arrival counters of the decode path).
+__global__ void __launch_bounds__(1024) indexer_prep_kernel(const int32_t* __restrict__ tok_seq,
                                                             const int32_t* __restrict__ tok_pos,
                                                             int32_t T, int32_t batch,
                                                             int32_t max_pos, int32_t pos_cap,
-                                                            void* ws) {
+                                                            void* ws, uint32_t* zero,
+                                                            int64_t zero_words) {
   __shared__ int sm[33];
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t i = threadIdx.x; i < zero_words; i += blockDim.x) zero[i] = 0u;
   PlanView v = plan_view(ws, T);
   const int n_groups = (T + kRunTokens - 1) / kRunTokens;
   int carry = 0;
@@ -172,6 +178,7 @@ struct IdxArgs {
   int64_t ld;
   void* plan;
   int32_t T;
+  uint32_t* hist;  // [T][2048] first-digit histogram of the ordered logits, or null
 };
 
 __host__ __device__ constexpr int pow2ceil(int x) {
@@ -191,8 +198,9 @@ struct IdxCfg {
   static constexpr int kOffQ = kOffK + kStages * kTileBytes;
   static constexpr int kOffWq = kOffQ + 2 * kQBytes;
   static constexpr int kOffMeta = kOffWq + 2 * kRunTokens * HP * 4;
-  static constexpr int kOffBar = kOffMeta + 64;
-  static constexpr int kNumBars = 2 * kStages + 9;
+  static constexpr int kOffHist = kOffMeta + 64;
+  static constexpr int kOffBar = kOffHist + kRunTokens * 2048 * 4;
+  static constexpr int kNumBars = 2 * kStages + 11;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16;
   static constexpr int kSmemAlloc = kSmem + 1024;
@@ -249,10 +257,14 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tfull = qempty + 2;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
+  uint64_t* hist_full = drain + 1;
+  uint64_t* hist_free = drain + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();  // the plan (and the zeroed histogram) come from the prep kernel
+  pdl_trigger();
   PlanView pv = plan_view(a.plan, a.T);
   const int n_runs = pv.hdr[0];
   const int total = pv.hdr[1];
@@ -272,6 +284,8 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&tempty[q], 4);
     }
     mbar_init(drain, 1);
+    mbar_init(hist_full, 4);
+    mbar_init(hist_free, 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -279,6 +293,9 @@ __global__ void __launch_bounds__(192, 1)
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
+  uint32_t* shist = reinterpret_cast<uint32_t*>(smem + C::kOffHist);
+  if (a.hist)
+    for (int i = threadIdx.x; i < kRunTokens * 2048; i += blockDim.x) shist[i] = 0u;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -392,7 +409,7 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    int n = 0;
+    int n = 0, n_flush = 0;
     int slot = 0;
     for (; wk.next(); wk.advance(), ++n) {
       const int r = wk.r;
@@ -430,8 +447,9 @@ __global__ void __launch_bounds__(192, 1)
             acc0 = fmaf(fmaxf(x[h], 0.f), wv[h], acc0);
             acc1 = fmaf(fmaxf(x[h + 1], 0.f), wv[h + 1], acc1);
           }
-          a.logits[static_cast<int64_t>(qtok[slot * kRunTokens + j]) * a.ld + s] =
-              (acc0 + acc1) * ks;
+          const float v = (acc0 + acc1) * ks;
+          a.logits[static_cast<int64_t>(qtok[slot * kRunTokens + j]) * a.ld + s] = v;
+          if (a.hist) atomicAdd(&shist[j * 2048 + (float_to_ordered(v) >> 21)], 1u);
         }
       }
       tc_fence_before();
@@ -439,6 +457,28 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) {
         mbar_arrive(&tempty[ab]);
         if (wk.last_of_run) mbar_arrive(&qempty[slot]);
+      }
+      if (a.hist && wk.last_of_run) {
+        // this CTA is done with the run: add its histogram to the global one.  The four
+        // epilogue warps meet on hist_full, each flushes (and clears) a quarter of the
+        // bins, and they meet again on hist_free before any bin is reused.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(hist_full);
+        if (!mbar_wait(hist_full, n_flush & 1, abort_flag)) break;
+        for (int j = 0; j < ntok; ++j) {
+          uint32_t* gh = a.hist + static_cast<size_t>(qtok[slot * kRunTokens + j]) * 2048;
+          for (int d = quarter * 512 + lane; d < (quarter + 1) * 512; d += 32) {
+            const uint32_t c = shist[j * 2048 + d];
+            if (c) {
+              atomicAdd(&gh[d], c);
+              shist[j * 2048 + d] = 0u;
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(hist_free);
+        if (!mbar_wait(hist_free, n_flush & 1, abort_flag)) break;
+        ++n_flush;
       }
     }
   }
@@ -468,13 +508,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 template <int DI, int HP>
 static cudaError_t launch_indexer_t(const IndexerLaunch& L, const CUtensorMap& map, int grid) {
   using C = IdxCfg<DI, HP>;
-  static bool attr_set = false;  // per process; the attribute is per function, all devices
-  if (!attr_set) {
+  static int attr_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
     cudaError_t e = cudaFuncSetAttribute(indexer_kernel<DI, HP>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemAlloc);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_dev = dev;
   }
   IdxArgs a;
   a.k_scale = L.cache->k_scale;
@@ -490,9 +532,9 @@ static cudaError_t launch_indexer_t(const IndexerLaunch& L, const CUtensorMap& m
   a.ld = L.ld_logits;
   a.plan = L.ws;
   a.T = L.queries->n_tokens;
-  indexer_kernel<DI, HP><<<grid, 192, C::kSmemAlloc, L.stream>>>(map, a);
-  count_launch();
-  return cudaGetLastError();
+  a.hist = L.hist;
+  return launch_pdl(indexer_kernel<DI, HP>, dim3(grid), dim3(192), C::kSmemAlloc, L.stream, map,
+                    a);
 }
 
 cudaError_t launch_indexer(const IndexerLaunch& L) {
@@ -500,10 +542,9 @@ cudaError_t launch_indexer(const IndexerLaunch& L) {
   const dsa_queries* q = L.queries;
   const int T = q->n_tokens;
   if (T == 0) return cudaSuccess;
-  indexer_plan_kernel<<<1, 1024, 0, L.stream>>>(q->tok_seq, q->tok_pos, T, c->batch, q->max_pos,
-                                                c->max_blocks_per_seq * kPage, L.ws);
-  count_launch();
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(indexer_prep_kernel, dim3(1), dim3(1024), 0, L.stream, q->tok_seq,
+                             q->tok_pos, T, c->batch, q->max_pos, c->max_blocks_per_seq * kPage,
+                             L.ws, L.zero, L.zero_words);
   if (e != cudaSuccess) return e;
 
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();

@@ -22,10 +22,14 @@ constexpr int kTopkThreads = 1024;
 constexpr int kTopkCand = 8192;       // threshold-bucket candidates kept in shared memory
 constexpr int kTopkRowCache = 32768;  // rows up to this length are cached in shared memory
 
+constexpr int kTopkMaxChunks = 128;  // CTAs per row in the decode variant
+
 struct TopkSmem {
   uint32_t hist[2048];
   int scan[72];
   int sel[4];
+  int pre_a[kTopkMaxChunks + 1];
+  int pre_b[kTopkMaxChunks + 1];
   uint32_t cand_key[kTopkCand];
   int32_t cand_idx[kTopkCand];
 };
@@ -38,6 +42,18 @@ struct RowGlobal {
   const float* row;
   __device__ uint32_t key(int i) const { return float_to_ordered(row[i]); }
   __device__ int index(int i) const { return i; }
+};
+struct RowGlobalOff {
+  const float* row;
+  int off;
+  __device__ uint32_t key(int i) const { return float_to_ordered(row[off + i]); }
+  __device__ int index(int i) const { return off + i; }
+};
+struct CandGlobal {
+  const float* row;
+  const int32_t* list;
+  __device__ uint32_t key(int i) const { return float_to_ordered(row[list[i]]); }
+  __device__ int index(int i) const { return list[i]; }
 };
 struct RowCached {
   const uint32_t* keys;
@@ -68,7 +84,8 @@ __device__ __forceinline__ void scan_two(TopkSmem* sm, int wa, int wb, int* off_
   }
   __syncthreads();
   if (wid == 0) {
-    int a = sm->scan[lane], b = sm->scan[32 + lane];
+    const bool live = lane < static_cast<int>(blockDim.x >> 5);
+    int a = live ? sm->scan[lane] : 0, b = live ? sm->scan[32 + lane] : 0;
     int ia = a, ib = b;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -119,15 +136,21 @@ __device__ void hist_pass(TopkSmem* sm, const Src& src, int n, int shift, int nb
 }
 
 // Largest bucket b with count(> b) < k_rem <= count(>= b).  Writes sel[0] = b,
-// sel[1] = count(> b).
+// sel[1] = count(> b), sel[2] = count(b).  Thread t looks at `per` consecutive buckets in
+// descending order, starting at nb-1-t*per.
 __device__ void select_bucket(TopkSmem* sm, int nb, int k_rem) {
   const int t = threadIdx.x;
-  const int b0 = nb - 1 - 2 * t, b1 = b0 - 1;
-  const int c0 = b0 >= 0 ? static_cast<int>(sm->hist[b0]) : 0;
-  const int c1 = b1 >= 0 ? static_cast<int>(sm->hist[b1]) : 0;
-  // inclusive scan of (c0 + c1) in descending bucket order
+  const int per = (nb + blockDim.x - 1) / blockDim.x;  // 1, 2 or 4
+  int c[4];
+  int sum = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int b = nb - 1 - t * per - q;
+    c[q] = (q < per && b >= 0) ? static_cast<int>(sm->hist[b]) : 0;
+    sum += c[q];
+  }
   const int lane = t & 31, wid = t >> 5;
-  int x = c0 + c1;
+  int x = sum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -136,7 +159,7 @@ __device__ void select_bucket(TopkSmem* sm, int nb, int k_rem) {
   if (lane == 31) sm->scan[wid] = x;
   __syncthreads();
   if (wid == 0) {
-    const int v = sm->scan[lane];
+    const int v = lane < static_cast<int>(blockDim.x >> 5) ? sm->scan[lane] : 0;
     int iv = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -146,24 +169,24 @@ __device__ void select_bucket(TopkSmem* sm, int nb, int k_rem) {
     sm->scan[lane] = iv - v;
   }
   __syncthreads();
-  const int excl = sm->scan[wid] + x - (c0 + c1);
-  if (b0 >= 0 && excl < k_rem && excl + c0 >= k_rem) {
-    sm->sel[0] = b0;
-    sm->sel[1] = excl;
+  int run = sm->scan[wid] + x - sum;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int b = nb - 1 - t * per - q;
+    if (q < per && b >= 0 && run < k_rem && run + c[q] >= k_rem) {
+      sm->sel[0] = b;
+      sm->sel[1] = run;
+      sm->sel[2] = c[q];
+    }
+    run += c[q];
   }
-  if (b1 >= 0 && excl + c0 < k_rem && excl + c0 + c1 >= k_rem) {
-    sm->sel[0] = b1;
-    sm->sel[1] = excl + c0;
-    sm->sel[2] = c1;
-  }
-  if (b0 >= 0 && excl < k_rem && excl + c0 >= k_rem) sm->sel[2] = c0;
   __syncthreads();
 }
 
 // One ordered pass: class A elements go to outA[baseA + rank]; class B elements with
 // rank < limitB go to the B sink.  cls(key) -> 0 none, 1 A, 2 B.
 template <class Src, class Cls, class SinkB>
-__device__ void ordered_pass(TopkSmem* sm, const Src& src, int n, Cls cls, int32_t* outA,
+__device__ int2 ordered_pass(TopkSmem* sm, const Src& src, int n, Cls cls, int32_t* outA,
                              int baseA, SinkB sinkB, int limitB) {
   const int lane = threadIdx.x & 31;
   int run_a = 0, run_b = 0;
@@ -187,6 +210,26 @@ __device__ void ordered_pass(TopkSmem* sm, const Src& src, int n, Cls cls, int32
     run_a += tot_a;
     run_b += tot_b;
   }
+  return make_int2(run_a, run_b);
+}
+
+// Digits 2 and 3 over the threshold-bucket candidates of digit-1 bucket b1, then the
+// ordered output of the k2 entries they contribute, at out[0 .. k2).
+template <class Src>
+__device__ void finish_candidates(TopkSmem* sm, const Src& cs, int n_cand, uint32_t b1, int k2,
+                                  int32_t* out) {
+  hist_pass(sm, cs, n_cand, 10, 2048, 32, 0u);
+  select_bucket(sm, 2048, k2);
+  const uint32_t b2 = static_cast<uint32_t>(sm->sel[0]);
+  const int above2 = sm->sel[1];
+  hist_pass(sm, cs, n_cand, 0, 1024, 10, (b1 << 11) | b2);
+  select_bucket(sm, 1024, k2 - above2);
+  const uint32_t thr = (b1 << 21) | (b2 << 10) | static_cast<uint32_t>(sm->sel[0]);
+  const int need_eq = k2 - above2 - sm->sel[1];
+  int32_t* eq_out = out + (k2 - need_eq);
+  ordered_pass(
+      sm, cs, n_cand, [thr](uint32_t key) { return key > thr ? 1 : (key == thr ? 2 : 0); }, out,
+      0, [eq_out](int r, uint32_t, int idx) { eq_out[r] = idx; }, need_eq);
 }
 
 template <class Src>
@@ -201,27 +244,16 @@ __device__ void select_from(TopkSmem* sm, const Src& src, int n, int k, int32_t*
   if (n_cand <= kTopkCand) {
     // higher buckets are final; gather the threshold bucket in position order
     ordered_pass(
-        sm, src, n, [b1](uint32_t key) { return (key >> 21) > b1 ? 1 : ((key >> 21) == b1 ? 2 : 0); },
-        out, 0,
+        sm, src, n,
+        [b1](uint32_t key) { return (key >> 21) > b1 ? 1 : ((key >> 21) == b1 ? 2 : 0); }, out,
+        0,
         [sm](int r, uint32_t key, int idx) {
           sm->cand_key[r] = key;
           sm->cand_idx[r] = idx;
         },
         kTopkCand);
     __syncthreads();
-    RowCand cs{sm->cand_key, sm->cand_idx};
-    hist_pass(sm, cs, n_cand, 10, 2048, 32, 0u);
-    select_bucket(sm, 2048, k2);
-    const uint32_t b2 = static_cast<uint32_t>(sm->sel[0]);
-    const int above2 = sm->sel[1];
-    hist_pass(sm, cs, n_cand, 0, 1024, 10, (b1 << 11) | b2);
-    select_bucket(sm, 1024, k2 - above2);
-    const uint32_t thr = (b1 << 21) | (b2 << 10) | static_cast<uint32_t>(sm->sel[0]);
-    const int need_eq = k2 - above2 - sm->sel[1];
-    int32_t* eq_out = out + above1 + (k2 - need_eq);
-    ordered_pass(
-        sm, cs, n_cand, [thr](uint32_t key) { return key > thr ? 1 : (key == thr ? 2 : 0); },
-        out, above1, [eq_out](int r, uint32_t, int idx) { eq_out[r] = idx; }, need_eq);
+    finish_candidates(sm, RowCand{sm->cand_key, sm->cand_idx}, n_cand, b1, k2, out + above1);
   } else {
     hist_pass(sm, src, n, 10, 2048, 21, b1);
     select_bucket(sm, 2048, k2);
@@ -244,6 +276,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   extern __shared__ uint8_t topk_smem_raw[];
   TopkSmem* sm = reinterpret_cast<TopkSmem*>(topk_smem_raw);
   uint32_t* row_cache = reinterpret_cast<uint32_t*>(topk_smem_raw + kTopkSmemBase);
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   int32_t* out = idx + static_cast<int64_t>(t) * k;
   const int pos = tok_pos[t];
@@ -281,10 +315,179 @@ cudaError_t launch_topk(const float* logits, int64_t ld, const dsa_queries* q, i
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
-  topk_kernel<<<q->n_tokens, kTopkThreads, smem, stream>>>(logits, ld, q->tok_pos, q->max_pos, k,
-                                                           idx, cache_ok);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel, dim3(q->n_tokens), dim3(kTopkThreads), smem, stream, logits, ld,
+                    q->tok_pos, q->max_pos, k, idx, cache_ok);
+}
+
+// ---------------------------------------------------------------------------- decode variant
+// Few long rows (decode): the row is split over `chunks` CTAs.  The first radix digit comes
+// from the histogram the indexer built while writing the logits, so every CTA knows the
+// threshold bucket b1 at once.  Each CTA writes, in position order, its entries above b1
+// (final) and its entries in b1 (candidates) to scratch at its own position range and
+// posts the two counts; the last CTA to arrive (global counter, no waiting) concatenates
+// the finals in chunk order and resolves digits 2 and 3 over the candidates.  Output order
+// equals the single-CTA kernel's: finals ascending, then candidate winners ascending.
+constexpr int kTopkDecThreads = 512;
+
+struct TopkDecodeWs {
+  const uint32_t* hist;  // [T][2048] digit-1 histogram (from the indexer epilogue)
+  uint32_t* arrive;      // [T] arrival counters, zero on entry
+  int32_t* counts;       // [T][chunks][2]
+  int32_t* scr_a;        // [T][ld] finals, at each chunk's position range
+  int32_t* scr_b;        // [T][ld] candidates, same
+};
+
+__global__ void __launch_bounds__(kTopkDecThreads, 1)
+    topk_decode_kernel(const float* __restrict__ logits, int64_t ld,
+                       const int32_t* __restrict__ tok_pos, int32_t max_pos, int32_t k,
+                       int32_t* __restrict__ idx, TopkDecodeWs ws, int chunks) {
+  extern __shared__ uint8_t topk_smem_raw[];
+  TopkSmem* sm = reinterpret_cast<TopkSmem*>(topk_smem_raw);
+  pdl_wait();  // logits and histogram come from the indexer
+  pdl_trigger();
+  const int t = blockIdx.y, c = blockIdx.x;
+  int32_t* out = idx + static_cast<int64_t>(t) * k;
+  const int pos = tok_pos[t];
+  if (pos < 0 || pos > max_pos) {
+    if (c == 0) {
+      if (threadIdx.x == 0) record_error(kErrBadIndex);
+      for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
+    }
+    return;
+  }
+  const int n = pos + 1;
+  if (n <= k) {
+    if (c == 0)
+      for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = i < n ? i : -1;
+    return;
+  }
+  const float* row = logits + static_cast<int64_t>(t) * ld;
+  for (int b = threadIdx.x; b < 2048; b += blockDim.x)
+    sm->hist[b] = ws.hist[static_cast<size_t>(t) * 2048 + b];
+  __syncthreads();
+  select_bucket(sm, 2048, k);
+  const uint32_t b1 = static_cast<uint32_t>(sm->sel[0]);
+  const int above1 = sm->sel[1];
+  const int n_cand = sm->sel[2];
+  const int c0 = static_cast<int>(static_cast<int64_t>(n) * c / chunks);
+  const int c1 = static_cast<int>(static_cast<int64_t>(n) * (c + 1) / chunks);
+  int32_t* sa = ws.scr_a + static_cast<int64_t>(t) * ld;
+  int32_t* sb = ws.scr_b + static_cast<int64_t>(t) * ld;
+  const int2 cnt = ordered_pass(
+      sm, RowGlobalOff{row, c0}, c1 - c0,
+      [b1](uint32_t key) { return (key >> 21) > b1 ? 1 : ((key >> 21) == b1 ? 2 : 0); }, sa, c0,
+      [sb, c0](int r, uint32_t, int i) { sb[c0 + r] = i; }, c1 - c0);
+  if (threadIdx.x == 0) {
+    ws.counts[(static_cast<size_t>(t) * chunks + c) * 2] = cnt.x;
+    ws.counts[(static_cast<size_t>(t) * chunks + c) * 2 + 1] = cnt.y;
+    __threadfence();
+    const uint32_t prev = atomicAdd(&ws.arrive[t], 1u);
+    sm->sel[3] = (prev == static_cast<uint32_t>(chunks - 1)) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!sm->sel[3]) return;
+  __threadfence();
+  // ---- the last CTA of this row finishes it
+  if (threadIdx.x == 0) {
+    int pa = 0, pb = 0;
+    for (int cc = 0; cc < chunks; ++cc) {
+      sm->pre_a[cc] = pa;
+      sm->pre_b[cc] = pb;
+      pa += ws.counts[(static_cast<size_t>(t) * chunks + cc) * 2];
+      pb += ws.counts[(static_cast<size_t>(t) * chunks + cc) * 2 + 1];
+    }
+    sm->pre_a[chunks] = pa;
+    sm->pre_b[chunks] = pb;
+  }
+  __syncthreads();
+  for (int cc = 0; cc < chunks; ++cc) {
+    const int cs = static_cast<int>(static_cast<int64_t>(n) * cc / chunks);
+    const int na = sm->pre_a[cc + 1] - sm->pre_a[cc];
+    for (int i = threadIdx.x; i < na; i += blockDim.x) out[sm->pre_a[cc] + i] = sa[cs + i];
+  }
+  // the counts actually gathered decide (they equal the histogram's when all is well)
+  const int got_a = sm->pre_a[chunks], got_b = sm->pre_b[chunks];
+  const int k2 = k - got_a;
+  if (got_a != above1 || got_b != n_cand || k2 < 1 || k2 > got_b) {
+    if (threadIdx.x == 0) record_error(kErrBadIndex);
+    for (int i = got_a + threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
+    return;
+  }
+  if (got_b <= kTopkCand) {
+    for (int cc = 0; cc < chunks; ++cc) {
+      const int cs = static_cast<int>(static_cast<int64_t>(n) * cc / chunks);
+      const int nb = sm->pre_b[cc + 1] - sm->pre_b[cc];
+      for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        const int p = sb[cs + i];
+        sm->cand_idx[sm->pre_b[cc] + i] = p;
+        sm->cand_key[sm->pre_b[cc] + i] = float_to_ordered(row[p]);
+      }
+    }
+    __syncthreads();
+    finish_candidates(sm, RowCand{sm->cand_key, sm->cand_idx}, got_b, b1, k2, out + got_a);
+  } else {
+    // too many candidates for shared memory: compact them into the (now free) finals
+    // scratch and resolve from global memory
+    __syncthreads();
+    for (int cc = 0; cc < chunks; ++cc) {
+      const int cs = static_cast<int>(static_cast<int64_t>(n) * cc / chunks);
+      const int nb = sm->pre_b[cc + 1] - sm->pre_b[cc];
+      for (int i = threadIdx.x; i < nb; i += blockDim.x) sa[sm->pre_b[cc] + i] = sb[cs + i];
+    }
+    __threadfence_block();
+    __syncthreads();
+    finish_candidates(sm, CandGlobal{row, sa}, got_b, b1, k2, out + got_a);
+  }
+}
+
+size_t topk_decode_ws_bytes(int32_t T, int64_t ld, int chunks) {
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  return al(static_cast<size_t>(T) * 2048 * 4) + al(static_cast<size_t>(T) * 4) +
+         al(static_cast<size_t>(T) * chunks * 8) + 2 * al(static_cast<size_t>(T) * ld * 4);
+}
+
+int topk_decode_chunks(int32_t T, int32_t max_pos) {
+  int c = T > 0 ? num_sms() / T : 1;
+  const int by_len = (max_pos + 1) / 1024 + 1;
+  if (c > by_len) c = by_len;
+  if (c > kTopkMaxChunks) c = kTopkMaxChunks;
+  return c < 1 ? 1 : c;
+}
+
+TopkDecodeLayout topk_decode_layout(void* ws, int32_t T, int64_t ld, int chunks) {
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  TopkDecodeLayout L;
+  L.hist = reinterpret_cast<uint32_t*>(p);
+  p += al(static_cast<size_t>(T) * 2048 * 4);
+  L.arrive = reinterpret_cast<uint32_t*>(p);
+  p += al(static_cast<size_t>(T) * 4);
+  L.zero_words = (p - static_cast<uint8_t*>(ws)) / 4;
+  L.counts = reinterpret_cast<int32_t*>(p);
+  p += al(static_cast<size_t>(T) * chunks * 8);
+  L.scr_a = reinterpret_cast<int32_t*>(p);
+  p += al(static_cast<size_t>(T) * ld * 4);
+  L.scr_b = reinterpret_cast<int32_t*>(p);
+  return L;
+}
+
+cudaError_t launch_topk_decode(const float* logits, int64_t ld, const dsa_queries* q, int32_t k,
+                               int32_t* idx, const TopkDecodeLayout& L, int chunks,
+                               cudaStream_t stream) {
+  if (q->n_tokens == 0) return cudaSuccess;
+  static int attr_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
+    cudaError_t e = cudaFuncSetAttribute(topk_decode_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kTopkSmemBase));
+    if (e != cudaSuccess) return e;
+    attr_dev = dev;
+  }
+  TopkDecodeWs w{L.hist, L.arrive, L.counts, L.scr_a, L.scr_b};
+  return launch_pdl(topk_decode_kernel, dim3(chunks, q->n_tokens), dim3(kTopkDecThreads),
+                    kTopkSmemBase, stream, logits, ld, q->tok_pos, q->max_pos, k, idx, w, chunks);
 }
 
 }  // namespace dsa
