@@ -60,7 +60,7 @@ typedef enum {
  *   block_table[b * max_blocks_per_seq + s / page_size] * page_size + s % page_size.   */
 typedef struct {
   const uint8_t* k8;          /* device [num_blocks*page_size, idx_dim]  e4m3 index keys   */
-  const float* k_scale;       /* device [num_blocks*page_size]           per-token scale   */
+  const float* k_scale;       /* device [num_blocks*page_size]           per-token scale (16-B aligned) */
   const uint16_t* kv;         /* device [num_blocks*page_size, d_kv]     bf16 latent rows  */
   const int32_t* block_table; /* device [batch, max_blocks_per_seq]      physical blocks   */
   int32_t batch;              /* number of sequences                                       */
@@ -134,6 +134,17 @@ DSA_API size_t dsa_forward_workspace_size(int32_t n_tokens, int32_t max_pos, int
 /* Waits for `stream`, then returns and clears the device status word of the current
  * device (DSA_OK, DSA_ERR_BAD_INDEX or DSA_ERR_TIMEOUT; DSA_ERR_CUDA if the wait failed). */
 DSA_API dsa_status dsa_read_device_status(void* stream);
+
+/* Test hook for the failure path.  The next indexer launch (fault = 1) or attention launch
+ * (fault = 2) on this process skips one producer barrier arrival in its first CTA, so
+ * that CTA's bounded waits run out (after about 0.2 s), the kernel unwinds, and
+ * dsa_read_device_status() reports DSA_ERR_TIMEOUT; the CUDA context stays usable.
+ * fault = 0 clears a pending injection.  Nothing faults, traps or hangs.                */
+DSA_API dsa_status dsa_debug_inject(int32_t fault);
+
+/* Diagnosis of the last DSA_ERR_TIMEOUT that dsa_read_device_status() returned:
+ * 0x80000000 | (wait site << 16) | (blockIdx.x of the CTA), or 0 if none was recorded.   */
+DSA_API uint32_t dsa_debug_timeout_site(void);
 
 /* Number of kernel launches the library has enqueued in this process (all devices). */
 DSA_API int64_t dsa_launch_count(void);

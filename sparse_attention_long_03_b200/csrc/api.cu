@@ -9,9 +9,16 @@
 namespace dsa {
 
 __device__ uint32_t g_status = 0;
+__device__ uint32_t g_where = 0;
 
 static std::atomic<int64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static std::atomic<int> g_inject{0};
+int take_injection(int which) {
+  int expected = which;
+  return g_inject.compare_exchange_strong(expected, 0) ? 1 : 0;
+}
 
 int num_sms() {
   static int cached[64];
@@ -28,6 +35,7 @@ int num_sms() {
   return cached[dev];
 }
 
+extern uint32_t g_last_where;
 cudaError_t read_and_clear_status(cudaStream_t stream, uint32_t* out) {
   cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return e;
@@ -35,9 +43,17 @@ cudaError_t read_and_clear_status(cudaStream_t stream, uint32_t* out) {
   e = cudaMemcpyFromSymbol(&v, g_status, sizeof(v));
   if (e != cudaSuccess) return e;
   e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+  if (e != cudaSuccess) return e;
+  uint32_t where = 0;
+  e = cudaMemcpyFromSymbol(&where, g_where, sizeof(where));
+  if (e != cudaSuccess) return e;
+  g_last_where = where;
+  e = cudaMemcpyToSymbol(g_where, &zero, sizeof(zero));
   *out = v;
   return e;
 }
+
+uint32_t g_last_where = 0;
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -52,7 +68,7 @@ static dsa_status check_cache(const dsa_paged_cache* c, bool need_keys, bool nee
   if (need_keys) {
     if (!c->k8 || !c->k_scale) return DSA_ERR_INVALID_ARG;
     if (c->idx_dim != 32 && c->idx_dim != 64 && c->idx_dim != 128) return DSA_ERR_UNSUPPORTED;
-    if (!aligned(c->k8, 16) || !aligned(c->k_scale, 4)) return DSA_ERR_INVALID_ARG;
+    if (!aligned(c->k8, 16) || !aligned(c->k_scale, 16)) return DSA_ERR_INVALID_ARG;
   }
   if (need_kv) {
     if (!c->kv) return DSA_ERR_INVALID_ARG;
@@ -123,6 +139,14 @@ extern "C" {
 int32_t dsa_abi_version(void) { return 1; }
 
 int64_t dsa_launch_count(void) { return g_launches.load(); }
+
+uint32_t dsa_debug_timeout_site(void) { return g_last_where; }
+
+dsa_status dsa_debug_inject(int32_t fault) {
+  if (fault < 0 || fault > 2) return DSA_ERR_INVALID_ARG;
+  g_inject.store(fault);
+  return DSA_OK;
+}
 
 const char* dsa_status_string(dsa_status s) {
   switch (s) {

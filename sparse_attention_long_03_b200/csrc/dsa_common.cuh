@@ -34,9 +34,18 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
-// Every in-kernel wait gives up after this long (ns), records kErrTimeout and lets the
-// kernel unwind; no legitimate wait in these kernels lasts more than microseconds.
-constexpr uint64_t kWaitBudgetNs = 200ull * 1000ull * 1000ull;
+// Every in-kernel wait gives up after this many SM cycles (about 0.2-0.4 s between
+// 1.0 and 2.0 GHz), records kErrTimeout and lets the kernel unwind; no legitimate wait in
+// these kernels lasts more than microseconds.  SM cycles (clock64) always advance.
+constexpr long long kWaitBudgetCycles = 1ll << 29;
+
+// Where the first wait that gave up was: (site << 16) | (blockIdx.x & 0xffff), and the
+// phase parity it waited for; read by the host for diagnosis.
+extern __device__ uint32_t g_where;
+__device__ __forceinline__ void record_timeout(uint32_t site) {
+  record_error(2u);
+  atomicCAS(&g_where, 0u, (site << 16) | (blockIdx.x & 0xffffu) | 0x80000000u);
+}
 
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -87,34 +96,52 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
-// Bounded wait for the phase of parity `parity`.  On timeout: records kErrTimeout, sets
-// *abort (shared) and returns false.  Also returns false at once if *abort is set.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// Bounded wait for the phase of parity `parity`.  On timeout: records kErrTimeout and the
+// wait site, sets *abort (shared) and returns false.  Also returns false at once if
+// *abort is set.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t site = 0) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  const long long c0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitBudgetNs) {
-      record_error(kErrTimeout);
+    if (clock64() - c0 > kWaitBudgetCycles) {
+      record_timeout(site);
       *abort = 1;
       return false;
     }
   }
 }
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort) {
+                                                  volatile int* abort, uint32_t site = 0) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  const long long c0 = clock64();
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitBudgetNs) {
-      record_error(kErrTimeout);
+    if (clock64() - c0 > kWaitBudgetCycles) {
+      record_timeout(site);
       *abort = 1;
       return false;
     }
   }
+}
+// Warp-collective form: every lane of the warp polls, and all lanes get the same answer
+// (a lane that saw the phase complete while another gave up must not run on alone into
+// warp-synchronous instructions).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort, uint32_t site = 0) {
+  const bool ok = mbar_wait(bar, parity, abort, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait that ignores the abort flag (draining in-flight copies before exit).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const long long c0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - c0 > kWaitBudgetCycles) return false;
+  return true;
 }
 
 // ------------------------------------------------------------------ proxies / fences
@@ -129,6 +156,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+// Plain bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {

@@ -17,6 +17,8 @@ constexpr int kMaxTopK = 2048;
 
 void count_launch();
 int num_sms();
+// Pending test injection (see dsa_debug_inject); take_injection() consumes it.
+int take_injection(int which);
 
 // Launch `kernel` on `stream` with programmatic stream serialisation (the kernel may
 // overlap the tail of the previous kernel in the stream; it must call pdl_wait()).

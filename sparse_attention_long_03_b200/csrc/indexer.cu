@@ -179,6 +179,7 @@ struct IdxArgs {
   void* plan;
   int32_t T;
   uint32_t* hist;  // [T][2048] first-digit histogram of the ordered logits, or null
+  int inject;      // test hook: the CTA owning item 0 skips its first stage's arrival
 };
 
 __host__ __device__ constexpr int pow2ceil(int x) {
@@ -198,7 +199,9 @@ struct IdxCfg {
   static constexpr int kOffQ = kOffK + kStages * kTileBytes;
   static constexpr int kOffWq = kOffQ + 2 * kQBytes;
   static constexpr int kOffMeta = kOffWq + 2 * kRunTokens * HP * 4;
-  static constexpr int kOffHist = kOffMeta + 64;
+  static constexpr int kOffScale = kOffMeta + 64;                 // [S][128] fp32
+  static constexpr int kOffPage = kOffScale + kStages * kKeyTile * 4;  // [S][2] int32
+  static constexpr int kOffHist = kOffPage + kStages * 8 + 64;
   static constexpr int kOffBar = kOffHist + kRunTokens * 2048 * 4;
   static constexpr int kNumBars = 2 * kStages + 11;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -207,14 +210,6 @@ struct IdxCfg {
   static constexpr uint32_t kSwz = DI == 128 ? kSw128 : (DI == 64 ? kSw64 : kSw32);
   static_assert(kTileBytes % 1024 == 0 && kQBytes % 1024 == 0, "tile alignment");
 };
-
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitBudgetNs) return false;
-  }
-  return true;
-}
 
 // Walks this CTA's slice of the flat (run, tile) list in order; every role runs its
 // own copy so they agree on run boundaries without talking to each other.
@@ -261,21 +256,15 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* hist_free = drain + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  float* scales = reinterpret_cast<float*>(smem + C::kOffScale);
+  int* pages = reinterpret_cast<int*>(smem + C::kOffPage);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_wait();  // the plan (and the zeroed histogram) come from the prep kernel
-  pdl_trigger();
-  PlanView pv = plan_view(a.plan, a.T);
-  const int n_runs = pv.hdr[0];
-  const int total = pv.hdr[1];
-  const int i0 = static_cast<int>(static_cast<int64_t>(total) * blockIdx.x / gridDim.x);
-  const int i1 = static_cast<int>(static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x);
-  if (i0 >= i1) return;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 1 + 4);  // the MMA (keys) and the epilogue warps (scales)
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(&qfull[q], 1);
@@ -301,9 +290,17 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  pdl_wait();  // the plan (and the zeroed histogram) come from the prep kernel
+  pdl_trigger();
+  PlanView pv = plan_view(a.plan, a.T);
+  const int n_runs = pv.hdr[0];
+  const int total = pv.hdr[1];
+  const int i0 = static_cast<int>(static_cast<int64_t>(total) * blockIdx.x / gridDim.x);
+  const int i1 = static_cast<int>(static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x);
+
   // run containing item i0
   int lo = 0, hi = n_runs;  // item0[lo] <= i0 < item0[hi]
-  while (hi - lo > 1) {
+  while (i0 < i1 && hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (pv.item0[mid] <= i0) lo = mid;
     else hi = mid;
@@ -313,11 +310,12 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     int n = 0;
+    int bt_run = -1, bt_lb0 = 0, my_pb = -2;
     for (; wk.next(); wk.advance(), ++n) {
       const int r = wk.r;
       if (wk.new_run) {
         const int slot = wk.rc & 1;
-        if (!mbar_wait(&qempty[slot], ((wk.rc >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait_warp(&qempty[slot], ((wk.rc >> 1) & 1) ^ 1, abort_flag, 11)) break;
         const int tok0 = pv.tok0[r], ntok = pv.ntok[r];
         uint8_t* qb = qbuf + slot * C::kQBytes;
         constexpr int kChunks = DI / 16;
@@ -345,28 +343,40 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&qfull[slot]);
       }
+      // block-table entries, 32 pages per warp-wide load
+      if (r != bt_run || wk.tile * 2 < bt_lb0 || wk.tile * 2 + 1 >= bt_lb0 + 32) {
+        bt_run = r;
+        bt_lb0 = wk.tile * 2;
+        const int nblk = (pv.maxpos[r] + kPage) / kPage;
+        const int lb = bt_lb0 + lane;
+        my_pb = lb < nblk ? a.block_table[static_cast<size_t>(pv.seq[r]) * a.max_blocks + lb]
+                          : -2;  // -2: past the run's last block (not an error)
+      }
+      const int pb0 = __shfl_sync(0xffffffffu, my_pb, wk.tile * 2 - bt_lb0);
+      const int pb1 = __shfl_sync(0xffffffffu, my_pb, wk.tile * 2 + 1 - bt_lb0);
       const int stage = n % S;
-      if (!mbar_wait(&empty[stage], ((n / S) & 1) ^ 1, abort_flag)) break;
-      if (lane == 0) {
-        const int seq = pv.seq[r], nblk = (pv.maxpos[r] + kPage) / kPage;
-        int pb[2];
+      if (!mbar_wait_warp(&empty[stage], ((n / S) & 1) ^ 1, abort_flag, 12)) break;
+      if (lane == 0 && !(a.inject && i0 == 0 && n == 0)) {
+        int pb[2] = {pb0, pb1};
         uint32_t bytes = 0;
         for (int h = 0; h < 2; ++h) {
-          const int lb = wk.tile * 2 + h;
-          pb[h] = -1;
-          if (lb < nblk) {
-            const int p = a.block_table[static_cast<size_t>(seq) * a.max_blocks + lb];
-            if (p >= 0 && p < a.num_blocks) pb[h] = p;
-            else record_error(kErrBadIndex);
+          if (pb[h] != -2 && (pb[h] < 0 || pb[h] >= a.num_blocks)) {
+            record_error(kErrBadIndex);
+            pb[h] = -1;
           }
-          if (pb[h] >= 0) bytes += kPage * DI;
+          if (pb[h] == -2) pb[h] = -1;
+          pages[stage * 2 + h] = pb[h];
+          if (pb[h] >= 0) bytes += kPage * DI + kPage * 4;
         }
         if (bytes) mbar_arrive_expect_tx(&full[stage], bytes);
         else mbar_arrive(&full[stage]);
         for (int h = 0; h < 2; ++h)
-          if (pb[h] >= 0)
+          if (pb[h] >= 0) {
             tma_load_2d(ktiles + stage * C::kTileBytes + h * kPage * DI, &kmap, &full[stage], 0,
                         pb[h] * kPage);
+            bulk_load(scales + stage * kKeyTile + h * kPage,
+                      a.k_scale + static_cast<size_t>(pb[h]) * kPage, kPage * 4, &full[stage]);
+          }
       }
       __syncwarp();
     }
@@ -382,12 +392,12 @@ __global__ void __launch_bounds__(192, 1)
         const int r = wk.r;
         if (wk.new_run) {
           slot = wk.rc & 1;
-          if (!mbar_wait(&qfull[slot], (wk.rc >> 1) & 1, abort_flag)) break;
+          if (!mbar_wait(&qfull[slot], (wk.rc >> 1) & 1, abort_flag, 13)) break;
         }
         const int ab = n & 1;
-        if (!mbar_wait(&tempty[ab], ((n >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(&tempty[ab], ((n >> 1) & 1) ^ 1, abort_flag, 14)) break;
         const int stage = n % S;
-        if (!mbar_wait(&full[stage], (n / S) & 1, abort_flag)) break;
+        if (!mbar_wait(&full[stage], (n / S) & 1, abort_flag, 15)) break;
         tc_fence_after();
         const uint32_t N = static_cast<uint32_t>(pv.ntok[r] * HP);
         const uint32_t idesc = instr_desc(128, N, 0, 0, 0, 0);
@@ -415,19 +425,18 @@ __global__ void __launch_bounds__(192, 1)
       const int r = wk.r;
       if (wk.new_run) {
         slot = wk.rc & 1;
-        if (!mbar_wait(&qfull[slot], (wk.rc >> 1) & 1, abort_flag)) break;
+        if (!mbar_wait_warp(&qfull[slot], (wk.rc >> 1) & 1, abort_flag, 16)) break;
       }
       const int ab = n & 1;
-      if (!mbar_wait(&tfull[ab], (n >> 1) & 1, abort_flag)) break;
+      if (!mbar_wait_warp(&tfull[ab], (n >> 1) & 1, abort_flag, 17)) break;
       tc_fence_after();
       const int s = wk.tile * kKeyTile + row;
       const int ntok = pv.ntok[r];
-      float ks = __int_as_float(0x7fc00000);
-      if (s <= pv.maxpos[r]) {
-        const int p =
-            a.block_table[static_cast<size_t>(pv.seq[r]) * a.max_blocks + s / kPage];
-        if (p >= 0 && p < a.num_blocks) ks = a.k_scale[static_cast<size_t>(p) * kPage + s % kPage];
-      }
+      const int stage = n % S;
+      // the stage's scales and page ids (complete: the MMA already waited for it)
+      if (!mbar_wait_warp(&full[stage], (n / S) & 1, abort_flag, 18)) break;
+      const float ks = pages[stage * 2 + (row >> 6)] >= 0 ? scales[stage * kKeyTile + row]
+                                                           : __int_as_float(0x7fc00000);
       for (int j = 0; j < ntok; ++j) {
         float x[HP];
         const uint32_t taddr =
@@ -456,6 +465,7 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&tempty[ab]);
+        mbar_arrive(&empty[stage]);
         if (wk.last_of_run) mbar_arrive(&qempty[slot]);
       }
       if (a.hist && wk.last_of_run) {
@@ -464,7 +474,7 @@ __global__ void __launch_bounds__(192, 1)
         // bins, and they meet again on hist_free before any bin is reused.
         __syncwarp();
         if (lane == 0) mbar_arrive(hist_full);
-        if (!mbar_wait(hist_full, n_flush & 1, abort_flag)) break;
+        if (!mbar_wait_warp(hist_full, n_flush & 1, abort_flag, 19)) break;
         for (int j = 0; j < ntok; ++j) {
           uint32_t* gh = a.hist + static_cast<size_t>(qtok[slot * kRunTokens + j]) * 2048;
           for (int d = quarter * 512 + lane; d < (quarter + 1) * 512; d += 32) {
@@ -477,7 +487,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(hist_free);
-        if (!mbar_wait(hist_free, n_flush & 1, abort_flag)) break;
+        if (!mbar_wait_warp(hist_free, n_flush & 1, abort_flag, 20)) break;
         ++n_flush;
       }
     }
@@ -533,6 +543,7 @@ static cudaError_t launch_indexer_t(const IndexerLaunch& L, const CUtensorMap& m
   a.plan = L.ws;
   a.T = L.queries->n_tokens;
   a.hist = L.hist;
+  a.inject = take_injection(1);
   return launch_pdl(indexer_kernel<DI, HP>, dim3(grid), dim3(192), C::kSmemAlloc, L.stream, map,
                     a);
 }

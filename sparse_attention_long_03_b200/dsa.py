@@ -27,7 +27,8 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
 EXPORTED = ("dsa_indexer_logits", "dsa_indexer_workspace_size", "dsa_topk",
             "dsa_topk_workspace_size", "dsa_sparse_mla_attn", "dsa_attn_workspace_size",
             "dsa_forward", "dsa_forward_workspace_size", "dsa_read_device_status",
-            "dsa_launch_count", "dsa_status_string", "dsa_abi_version")
+            "dsa_launch_count", "dsa_status_string", "dsa_abi_version", "dsa_debug_inject",
+            "dsa_debug_timeout_site")
 
 
 class DsaError(RuntimeError):
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
             "dsa_launch_count": (I64, []),
             "dsa_status_string": (ctypes.c_char_p, [I32]),
             "dsa_abi_version": (I32, []),
+            "dsa_debug_inject": (I32, [I32]),
+            "dsa_debug_timeout_site": (ctypes.c_uint32, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -204,3 +207,13 @@ def dsa_read_device_status(stream=None) -> int:
 
 def dsa_launch_count() -> int:
     return int(lib().dsa_launch_count())
+
+
+def dsa_debug_timeout_site() -> int:
+    """Site of the last timeout read by dsa_read_device_status (0 if none)."""
+    return int(lib().dsa_debug_timeout_site())
+
+
+def dsa_debug_inject(fault: int) -> None:
+    """Test hook: make the next indexer (1) or attention (2) launch time out on purpose."""
+    _check("dsa_debug_inject", lib().dsa_debug_inject(int(fault)))
