@@ -95,6 +95,22 @@ DSA_API dsa_status dsa_indexer_logits(const dsa_paged_cache* cache, const dsa_qu
                               void* workspace, size_t workspace_bytes, void* stream);
 DSA_API size_t dsa_indexer_workspace_size(int32_t n_tokens);
 
+/* dsa_indexer_logits for callers that cannot allocate device memory (a plugin host that
+ * passes only input and output pointers, a runtime that forbids allocation after
+ * start-up, a foreign-function binding without a device allocator).  It has no
+ * counterpart in the paper: it is the same computation, with the scratch taken from a
+ * 256 KiB array that the library keeps in device memory on every GPU that loads it, for
+ * calls of at most 12288 query tokens (more: DSA_ERR_WORKSPACE, nothing launched).  All
+ * calls share that array, so calls whose kernels overlap on the GPU race; calls ordered
+ * on one stream are fine.  The first call on a device looks up the array's address and
+ * should come before any stream capture starts.  Other arguments, results and errors are
+ * those of dsa_indexer_logits.                                                            */
+DSA_API dsa_status dsa_indexer_logits_noalloc(const dsa_paged_cache* cache,
+                                              const dsa_queries* queries, const uint8_t* q8,
+                                              const float* q_scale, const float* w,
+                                              int32_t n_idx_heads, float* logits,
+                                              int64_t ld_logits, void* stream);
+
 /* (2) Per-row top-k by radix select (no sort) over logits[t, 0..tok_pos[t]].
  * idx  device [T, k] int32: the logical positions of the min(k, tok_pos[t]+1) largest
  *      logits of row t (equal values: the smaller position first), -1 in unused slots.

@@ -1,0 +1,81 @@
+// dsa_indexer_logits_noalloc: the lightning indexer for callers that cannot allocate
+// device memory.
+//
+// dsa_indexer_logits needs a small scratch buffer (the work plan: which query tokens share
+// a key tile and where each CTA's slice of the work starts).  Normally the caller passes
+// it in.  Some callers have no way to get device memory: a plugin host that hands the
+// library nothing but its input and output pointers, a runtime that forbids allocation
+// once it has started (fixed memory budgets, real-time loops), or a foreign-function
+// binding with no device allocator in reach.  For them this entry point keeps the scratch
+// in a fixed array in the library's own device memory.
+//
+// Costs and limits of that choice:
+//   * the array is kStaticScratchBytes (256 KiB) on every GPU that loads the library, held
+//     until the process exits; it fits calls with at most kStaticMaxTokens query tokens;
+//     larger calls are rejected with DSA_ERR_WORKSPACE before anything is launched;
+//   * every call shares the one array: two calls whose kernels overlap on the GPU (on
+//     different streams, say) race on it and give wrong results.  Calls on one stream, or
+//     otherwise ordered, are fine;
+//   * the array keeps whatever the last call left in it; nothing here needs it to start
+//     at zero, because the planner writes every word the indexer then reads;
+//   * the first call on each device looks up the array's device address (with that device
+//     current) and caches it; make that first call before any stream capture begins.
+#include <mutex>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int32_t kStaticMaxTokens = 12288;
+constexpr size_t kStaticScratchBytes = 256 * 1024;
+// the plan of kStaticMaxTokens tokens: header, five per-token arrays and one extra word
+static_assert(((4 + 5 * static_cast<size_t>(kStaticMaxTokens) + 1) * 4 + 255) / 256 * 256 <=
+                  kStaticScratchBytes,
+              "static indexer scratch too small for its stated maximum");
+
+// Device memory owned by the library.  In host code this name is only a host-side handle
+// for the symbol, not a device address: the address a kernel may use comes from
+// cudaGetSymbolAddress below.
+__device__ __align__(256) uint8_t g_indexer_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mutex;
+
+// Device address of the scratch array on the current device (looked up once per device).
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_indexer_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace dsa
+
+extern "C" dsa_status dsa_indexer_logits_noalloc(const dsa_paged_cache* cache,
+                                                 const dsa_queries* queries, const uint8_t* q8,
+                                                 const float* q_scale, const float* w,
+                                                 int32_t n_idx_heads, float* logits,
+                                                 int64_t ld_logits, void* stream) {
+  if (!queries) return DSA_ERR_INVALID_ARG;
+  if (queries->n_tokens > dsa::kStaticMaxTokens) return DSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (dsa::scratch_address(&scratch) != cudaSuccess) {
+    cudaGetLastError();
+    return DSA_ERR_CUDA;
+  }
+  return dsa_indexer_logits(cache, queries, q8, q_scale, w, n_idx_heads, logits, ld_logits,
+                            scratch, dsa::kStaticScratchBytes, stream);
+}

@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_WORKSPACE", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_BAD_INDEX",
                 6: "DSA_ERR_TIMEOUT"}
 
-EXPORTED = ("dsa_indexer_logits", "dsa_indexer_workspace_size", "dsa_topk",
+EXPORTED = ("dsa_indexer_logits", "dsa_indexer_workspace_size", "dsa_indexer_logits_noalloc",
+            "dsa_topk",
             "dsa_topk_workspace_size", "dsa_sparse_mla_attn", "dsa_attn_workspace_size",
             "dsa_forward", "dsa_forward_workspace_size", "dsa_read_device_status",
             "dsa_launch_count", "dsa_status_string", "dsa_abi_version", "dsa_debug_inject",
@@ -75,6 +76,7 @@ def lib() -> ctypes.CDLL:
         sig = {
             "dsa_indexer_logits": (I32, [PC, PQ, P, P, P, I32, P, I64, P, SZ, P]),
             "dsa_indexer_workspace_size": (SZ, [I32]),
+            "dsa_indexer_logits_noalloc": (I32, [PC, PQ, P, P, P, I32, P, I64, P]),
             "dsa_topk": (I32, [P, I64, PQ, I32, P, P, SZ, P]),
             "dsa_topk_workspace_size": (SZ, [I32, I32, I32]),
             "dsa_sparse_mla_attn": (I32, [PC, PQ, P, I32, I32, F32, P, I32, P, P, P, SZ, P]),
@@ -150,6 +152,18 @@ def dsa_indexer_logits(cache: PagedCache, queries: Queries, q8, q_scale, w, logi
                                   logits.shape[1], _ptr(workspace), workspace.numel(),
                                   _stream(stream))
     _check("dsa_indexer_logits", st)
+    return logits
+
+
+def dsa_indexer_logits_noalloc(cache: PagedCache, queries: Queries, q8, q_scale, w, logits,
+                               stream=None):
+    """dsa_indexer_logits without a workspace argument, for callers that cannot allocate
+    device memory: the library uses its own fixed 256 KiB device array (at most 12288
+    query tokens per call; calls that overlap on the GPU share it and race)."""
+    st = lib().dsa_indexer_logits_noalloc(ctypes.byref(cache), ctypes.byref(queries), _ptr(q8),
+                                          _ptr(q_scale), _ptr(w), q8.shape[1], _ptr(logits),
+                                          logits.shape[1], _stream(stream))
+    _check("dsa_indexer_logits_noalloc", st)
     return logits
 
 
