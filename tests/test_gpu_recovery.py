@@ -36,8 +36,9 @@ def test_indexer_timeout_is_reported_and_recovered():
     assert time.time() - t0 < 10.0
     again = w.indexer()
     assert dsa.dsa_read_device_status() == 0
-    n = int(w.host_q.tok_pos.max()) + 1
-    assert torch.equal(again[:, :n], ref[:, :n])
+    for t in range(w.host_q.n_tokens):  # entries past a token's position are not written
+        n = int(w.host_q.tok_pos[t]) + 1
+        assert torch.equal(again[t, :n], ref[t, :n])
 
 
 def test_attention_timeout_is_reported_and_recovered():
