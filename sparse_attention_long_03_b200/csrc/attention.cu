@@ -12,18 +12,19 @@
 // (128 heads x 512 fp32) would fill all of TMEM, so the value dims are split over G = 2
 // CTAs (value groups) that each own 256 of them; each computes the full 576-wide scores
 // itself (tcgen05, BF16, fp32 in TMEM, double-buffered) and runs the same online softmax.
-// Loads are TMA only: the query as 64-dim chunks (box 128 x 64), the selected latent rows
-// one row per copy (box 1 x 64) straight from the paged cache through the block table,
-// into a ring of (query chunk, key chunk) slots for the scores and a double-buffered
+// The query arrives by TMA as 64-dim chunks (box 128 x 64); the selected latent rows are
+// gathered through the block table by three producer warps with 16-byte vector loads and
+// swizzled shared-memory stores (empty slots become zeros), into a ring of (query chunk,
+// key chunk) slots for the scores (one slot per producer warp) and a double-buffered
 // value buffer for P.V (P as two bf16 parts hi + lo in shared memory, the A operand, so
 // the probabilities keep ~16 significant bits; V: an MN-major B operand, one 64-dim atom
 // per MMA).  Rescaling of O is lazy: the running max used for P
 // only moves when it grows by more than 2^8.  Long selections are split over several CTAs
 // (split-KV) and merged by LSE in a second kernel.
 //
-//   warp 0      producer: TMA copies (query chunks, selected rows)
-//   warp 1      one thread issues tcgen05.mma for S and for P.V, and the commits
-//   warps 2..5  softmax: online softmax, P, O rescale, output
+//   warps 0..3  softmax: online softmax, P, O rescale, output (one head row per thread)
+//   warp 4      one thread issues tcgen05.mma for S and for P.V, and the commits
+//   warps 5..7  producers: query-chunk TMA, row gathers into the ring and value buffer
 #include <cudaTypedefs.h>
 
 #include "dsa_common.cuh"
@@ -33,7 +34,7 @@ namespace dsa {
 
 namespace attn {
 constexpr int kBN = 64;                    // keys per tile
-constexpr int kRing = 4;                   // (query chunk, key chunk) slots
+constexpr int kRing = 3;                   // (query chunk, key chunk) slots, one per producer
 constexpr int kQChunk = 128 * 128;         // 128 heads x 64 bf16
 constexpr int kKVChunk = kBN * 128;        // 64 keys x 64 bf16
 constexpr int kSlot = kQChunk + kKVChunk;  // 24 KB
@@ -55,6 +56,7 @@ static_assert(kSlot % 1024 == 0 && kVBuf % 1024 == 0, "swizzle atoms");
 }  // namespace attn
 
 struct AttnArgs {
+  const uint16_t* kv;  // latent cache [num_blocks * 64, d_kv] bf16
   const int32_t* block_table;
   int32_t max_blocks;
   int32_t num_blocks;
@@ -93,9 +95,11 @@ __device__ __forceinline__ int resolve_row(int v, int pos, int seq, const AttnAr
   return p * kPage + v % kPage;
 }
 
-__global__ void __launch_bounds__(192, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap,
-                      const __grid_constant__ CUtensorMap kvmap, const AttnArgs a) {
+constexpr int kProducers = 3;  // producer warps 5..7
+constexpr int kAttnThreads = (5 + kProducers) * 32;
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap, const AttnArgs a) {
   using namespace attn;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -130,11 +134,11 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kRing; ++i) {
-      mbar_init(&ring_full[i], 1);
+      mbar_init(&ring_full[i], 1 + 32);  // the query TMA's expect_tx + the 32 gathering lanes
       mbar_init(&ring_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&v_full[i], 1);
+      mbar_init(&v_full[i], kProducers * 32);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
@@ -145,15 +149,9 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0) {
+  if (warp == 4) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
-  }
-  if (warp >= 2) {
-    // value rows of empty slots are never loaded: keep them finite (P is 0 there)
-    uint4* z = reinterpret_cast<uint4*>(vbuf);
-    for (int i = threadIdx.x - 64; i < 2 * kVBuf / 16; i += 128) z[i] = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -161,64 +159,94 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tmem_o = tmem + 2 * kBN;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    prefetch_tmap(&qmap);
-    prefetch_tmap(&kvmap);
-    int ring_n = 0, v_n = 0;
+  if (warp >= 5) {
+    // ---------------------------------------------------------------- producers
+    const int pw = warp - 5;  // owns ring slot pw and every kProducers-th piece of a V tile
+    if (lane == 0) prefetch_tmap(&qmap);
+    int ring_n = 0, q_issued = 0, last_slot_n = -1;
     bool ok = true;
     for (int i = 0; ok && i < n_tiles; ++i) {
+      // physical rows of the tile's 64 slots: lane l resolves slots l and l + 32
       int rows[2];
       for (int u = 0; u < 2; ++u) {
         const int slot = k0 + i * kBN + lane + 32 * u;
         const int v = slot < k1 ? a.idx[static_cast<size_t>(t) * a.k + slot] : -1;
-        rows[u] = resolve_row(v, pos, seq, a, true);
+        rows[u] = resolve_row(v, pos, seq, a, pw == 0);
       }
-      const int nvalid = __popc(__ballot_sync(0xffffffffu, rows[0] >= 0)) +
-                         __popc(__ballot_sync(0xffffffffu, rows[1] >= 0));
-      // score operands: query chunk c and key chunk c of this tile, chunk by chunk
-      for (int c = 0; c < nc; ++c) {
-        const int slot = ring_n % kRing;
-        if (!mbar_wait_warp(&ring_empty[slot], ((ring_n / kRing) & 1) ^ 1, abort_flag, 41)) {
+      // score operands: chunk c goes to ring slot n % kRing, filled by warp n % kRing
+      for (int c = 0; c < nc; ++c, ++ring_n) {
+        if (ring_n % kRing != pw) continue;
+        if (!mbar_wait_warp(&ring_empty[pw], ((ring_n / kRing) & 1) ^ 1, abort_flag, 41)) {
           ok = false;
           break;
         }
-        uint8_t* sb = ring + slot * kSlot;
+        uint8_t* sb = ring + pw * kSlot;
         if (lane == 0 && !(a.inject && blockIdx.x == 0 && blockIdx.y == 0 && ring_n == 0)) {
-          mbar_arrive_expect_tx(&ring_full[slot], kQChunk + nvalid * 128);
-          tma_load_2d(sb, &qmap, &ring_full[slot], c * 64, t * a.H);
+          mbar_arrive_expect_tx(&ring_full[pw], kQChunk);
+          tma_load_2d(sb, &qmap, &ring_full[pw], c * 64, t * a.H);
+          ++q_issued;
         }
-        __syncwarp();
-        for (int u = 0; u < 2; ++u)
-          if (rows[u] >= 0)
-            tma_load_2d(sb + kQChunk + (lane + 32 * u) * 128, &kvmap, &ring_full[slot], c * 64,
-                        rows[u]);
-        ++ring_n;
+        last_slot_n = ring_n;
+        // 64 rows x 8 pieces of 16 B: lane handles pieces lane + 32 j, 8 loads in flight
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint4 v[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int p = lane + 32 * (8 * half + j), r = p >> 3, c16 = p & 7;
+            const int r0 = __shfl_sync(0xffffffffu, rows[0], r & 31);
+            const int r1 = __shfl_sync(0xffffffffu, rows[1], r & 31);
+            const int row = (r >> 5) ? r1 : r0;
+            const int d0 = c * 64 + c16 * 8;
+            v[j] = (row >= 0 && d0 < a.d_kv) ? *reinterpret_cast<const uint4*>(
+                                                   a.kv + static_cast<size_t>(row) * a.d_kv + d0)
+                                             : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int p = lane + 32 * (8 * half + j), r = p >> 3, c16 = p & 7;
+            *reinterpret_cast<uint4*>(sb + kQChunk + swz_offset(r, c16 * 16, 128)) = v[j];
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&ring_full[pw]);
       }
       if (!ok) break;
-      // value chunks of this CTA for P.V
+      // this warp's share of the value tile: pieces lane + 32 j with j % kProducers == pw
       const int vb = i & 1;
       if (!mbar_wait_warp(&v_empty[vb], ((i >> 1) & 1) ^ 1, abort_flag, 42)) break;
-      if (lane == 0) {
-        if (nvalid) mbar_arrive_expect_tx(&v_full[vb], a.nvg * nvalid * 128);
-        else mbar_arrive(&v_full[vb]);
+      for (int vc = 0; vc < a.nvg; ++vc) {
+        uint4 v[6];
+#pragma unroll
+        for (int jj = 0; jj < 6; ++jj) {
+          const int j = pw + kProducers * jj;
+          if (j >= 16) break;
+          const int p = lane + 32 * j, r = p >> 3, c16 = p & 7;
+          const int r0 = __shfl_sync(0xffffffffu, rows[0], r & 31);
+          const int r1 = __shfl_sync(0xffffffffu, rows[1], r & 31);
+          const int row = (r >> 5) ? r1 : r0;
+          const int d0 = (vc0 + vc) * 64 + c16 * 8;
+          v[jj] = row >= 0 ? *reinterpret_cast<const uint4*>(a.kv + static_cast<size_t>(row) *
+                                                                         a.d_kv + d0)
+                           : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 6; ++jj) {
+          const int j = pw + kProducers * jj;
+          if (j >= 16) break;
+          const int p = lane + 32 * j, r = p >> 3, c16 = p & 7;
+          *reinterpret_cast<uint4*>(vbuf + vb * kVBuf + vc * kKVChunk +
+                                    swz_offset(r, c16 * 16, 128)) = v[jj];
+        }
       }
-      __syncwarp();
-      for (int vc = 0; vc < a.nvg; ++vc)
-        for (int u = 0; u < 2; ++u)
-          if (rows[u] >= 0)
-            tma_load_2d(vbuf + vb * kVBuf + vc * kKVChunk + (lane + 32 * u) * 128, &kvmap,
-                        &v_full[vb], (vc0 + vc) * 64, rows[u]);
-      v_n = i + 1;
+      fence_proxy_async_smem();
+      mbar_arrive(&v_full[vb]);
     }
-    // no copy may still be in flight when the CTA exits
-    if (lane == 0) {
-      for (int m = max(0, ring_n - kRing); m < ring_n; ++m)
-        mbar_wait_drain(&ring_full[m % kRing], (m / kRing) & 1);
-      for (int m = max(0, v_n - 2); m < v_n; ++m) mbar_wait_drain(&v_full[m & 1], (m >> 1) & 1);
-    }
+    // the last query TMA of this warp's slot must land before the CTA exits
+    if (lane == 0 && q_issued > 0 && last_slot_n >= 0)
+      mbar_wait_drain(&ring_full[pw], (last_slot_n / kRing) & 1);
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 4) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = instr_desc(128, kBN, 1, 1, 0, 0);
@@ -279,7 +307,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- softmax (warps 2..5)
+    // ---------------------------------------------------------------- softmax (warps 0..3)
     const int quarter = warp & 3;
     const int h = quarter * 32 + lane;  // head row == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -418,7 +446,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 4) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -538,12 +566,11 @@ cudaError_t launch_attn(const AttnLaunch& L) {
   const int tiles = (L.k + attn::kBN - 1) / attn::kBN;
   const int splits = attn_splits(T, L.k, groups);
   const int per_tiles = (tiles + splits - 1) / splits;
-  CUtensorMap qmap, kvmap;
-  if (!encode_rows(&qmap, L.q, static_cast<int64_t>(T) * L.n_heads, L.cache->d_kv, 128) ||
-      !encode_rows(&kvmap, L.cache->kv, static_cast<int64_t>(L.cache->num_blocks) * kPage,
-                   L.cache->d_kv, 1))
+  CUtensorMap qmap;
+  if (!encode_rows(&qmap, L.q, static_cast<int64_t>(T) * L.n_heads, L.cache->d_kv, 128))
     return cudaErrorInvalidValue;
   AttnArgs a;
+  a.kv = L.cache->kv;
   a.block_table = L.cache->block_table;
   a.max_blocks = L.cache->max_blocks_per_seq;
   a.num_blocks = L.cache->num_blocks;
@@ -570,8 +597,8 @@ cudaError_t launch_attn(const AttnLaunch& L) {
     a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(L.ws) +
                                           ((o + 255) & ~static_cast<size_t>(255)));
   }
-  sparse_mla_kernel<<<dim3(groups * splits, T), 192, attn::kSmemAlloc, L.stream>>>(qmap, kvmap,
-                                                                                  a);
+  sparse_mla_kernel<<<dim3(groups * splits, T), kAttnThreads, attn::kSmemAlloc, L.stream>>>(qmap,
+                                                                                           a);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || splits == 1) return e;

@@ -387,23 +387,36 @@ __global__ void __launch_bounds__(kTopkDecThreads, 1)
   __syncthreads();
   if (!sm->sel[3]) return;
   __threadfence();
-  // ---- the last CTA of this row finishes it
-  if (threadIdx.x == 0) {
-    int pa = 0, pb = 0;
-    for (int cc = 0; cc < chunks; ++cc) {
-      sm->pre_a[cc] = pa;
-      sm->pre_b[cc] = pb;
-      pa += ws.counts[(static_cast<size_t>(t) * chunks + cc) * 2];
-      pb += ws.counts[(static_cast<size_t>(t) * chunks + cc) * 2 + 1];
-    }
-    sm->pre_a[chunks] = pa;
-    sm->pre_b[chunks] = pb;
+  // ---- the last CTA of this row finishes it.  Every step below issues its global loads
+  // in parallel (no loop over chunks with a round trip per chunk).
+  for (int cc = threadIdx.x; cc < chunks; cc += blockDim.x) {
+    sm->pre_a[cc + 1] = ws.counts[(static_cast<size_t>(t) * chunks + cc) * 2];
+    sm->pre_b[cc + 1] = ws.counts[(static_cast<size_t>(t) * chunks + cc) * 2 + 1];
   }
   __syncthreads();
-  for (int cc = 0; cc < chunks; ++cc) {
-    const int cs = static_cast<int>(static_cast<int64_t>(n) * cc / chunks);
-    const int na = sm->pre_a[cc + 1] - sm->pre_a[cc];
-    for (int i = threadIdx.x; i < na; i += blockDim.x) out[sm->pre_a[cc] + i] = sa[cs + i];
+  if (threadIdx.x == 0) {
+    sm->pre_a[0] = 0;
+    sm->pre_b[0] = 0;
+    for (int cc = 0; cc < chunks; ++cc) {
+      sm->pre_a[cc + 1] += sm->pre_a[cc];
+      sm->pre_b[cc + 1] += sm->pre_b[cc];
+    }
+  }
+  __syncthreads();
+  // chunk holding flat entry g of a prefix array (largest cc with pre[cc] <= g)
+  auto chunk_of = [&](const int* pre, int g) {
+    int lo = 0, hi = chunks;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre[mid] <= g) lo = mid;
+      else hi = mid;
+    }
+    return lo;
+  };
+  auto chunk_start = [&](int cc) { return static_cast<int>(static_cast<int64_t>(n) * cc / chunks); };
+  for (int g = threadIdx.x; g < sm->pre_a[chunks]; g += blockDim.x) {
+    const int cc = chunk_of(sm->pre_a, g);
+    out[g] = sa[chunk_start(cc) + g - sm->pre_a[cc]];
   }
   // the counts actually gathered decide (they equal the histogram's when all is well)
   const int got_a = sm->pre_a[chunks], got_b = sm->pre_b[chunks];
@@ -414,14 +427,11 @@ __global__ void __launch_bounds__(kTopkDecThreads, 1)
     return;
   }
   if (got_b <= kTopkCand) {
-    for (int cc = 0; cc < chunks; ++cc) {
-      const int cs = static_cast<int>(static_cast<int64_t>(n) * cc / chunks);
-      const int nb = sm->pre_b[cc + 1] - sm->pre_b[cc];
-      for (int i = threadIdx.x; i < nb; i += blockDim.x) {
-        const int p = sb[cs + i];
-        sm->cand_idx[sm->pre_b[cc] + i] = p;
-        sm->cand_key[sm->pre_b[cc] + i] = float_to_ordered(row[p]);
-      }
+    for (int g = threadIdx.x; g < got_b; g += blockDim.x) {
+      const int cc = chunk_of(sm->pre_b, g);
+      const int p = sb[chunk_start(cc) + g - sm->pre_b[cc]];
+      sm->cand_idx[g] = p;
+      sm->cand_key[g] = float_to_ordered(row[p]);
     }
     __syncthreads();
     finish_candidates(sm, RowCand{sm->cand_key, sm->cand_idx}, got_b, b1, k2, out + got_a);
@@ -429,10 +439,9 @@ __global__ void __launch_bounds__(kTopkDecThreads, 1)
     // too many candidates for shared memory: compact them into the (now free) finals
     // scratch and resolve from global memory
     __syncthreads();
-    for (int cc = 0; cc < chunks; ++cc) {
-      const int cs = static_cast<int>(static_cast<int64_t>(n) * cc / chunks);
-      const int nb = sm->pre_b[cc + 1] - sm->pre_b[cc];
-      for (int i = threadIdx.x; i < nb; i += blockDim.x) sa[sm->pre_b[cc] + i] = sb[cs + i];
+    for (int g = threadIdx.x; g < got_b; g += blockDim.x) {
+      const int cc = chunk_of(sm->pre_b, g);
+      sa[g] = sb[chunk_start(cc) + g - sm->pre_b[cc]];
     }
     __threadfence_block();
     __syncthreads();
