@@ -162,6 +162,10 @@ DSA_API dsa_status dsa_debug_inject(int32_t fault);
  * 0x80000000 | (wait site << 16) | (blockIdx.x of the CTA), or 0 if none was recorded.   */
 DSA_API uint32_t dsa_debug_timeout_site(void);
 
+/* The cudaError_t code behind the last DSA_ERR_CUDA (or DSA_ERR_UNSUPPORTED from CUDA)
+ * any entry point returned in this process; 0 if none.                                   */
+DSA_API int32_t dsa_last_cuda_error(void);
+
 /* Number of kernel launches the library has enqueued in this process (all devices). */
 DSA_API int64_t dsa_launch_count(void);
 

@@ -84,8 +84,11 @@ static dsa_status check_queries(const dsa_queries* q) {
   return DSA_OK;
 }
 
+static std::atomic<int> g_last_cuda_error{0};
+
 static dsa_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return DSA_OK;
+  g_last_cuda_error.store(static_cast<int>(e));
   if (e == cudaErrorNotSupported) return DSA_ERR_UNSUPPORTED;
   cudaGetLastError();
   return DSA_ERR_CUDA;
@@ -141,6 +144,8 @@ int32_t dsa_abi_version(void) { return 1; }
 int64_t dsa_launch_count(void) { return g_launches.load(); }
 
 uint32_t dsa_debug_timeout_site(void) { return g_last_where; }
+
+int32_t dsa_last_cuda_error(void) { return g_last_cuda_error.load(); }
 
 dsa_status dsa_debug_inject(int32_t fault) {
   if (fault < 0 || fault > 2) return DSA_ERR_INVALID_ARG;

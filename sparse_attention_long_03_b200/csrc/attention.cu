@@ -12,19 +12,20 @@
 // (128 heads x 512 fp32) would fill all of TMEM, so the value dims are split over G = 2
 // CTAs (value groups) that each own 256 of them; each computes the full 576-wide scores
 // itself (tcgen05, BF16, fp32 in TMEM, double-buffered) and runs the same online softmax.
-// The query arrives by TMA as 64-dim chunks (box 128 x 64); the selected latent rows are
-// gathered through the block table by three producer warps with 16-byte vector loads and
-// swizzled shared-memory stores (empty slots become zeros), into a ring of (query chunk,
-// key chunk) slots for the scores (one slot per producer warp) and a double-buffered
-// value buffer for P.V (P as two bf16 parts hi + lo in shared memory, the A operand, so
-// the probabilities keep ~16 significant bits; V: an MN-major B operand, one 64-dim atom
-// per MMA).  Rescaling of O is lazy: the running max used for P
-// only moves when it grows by more than 2^8.  Long selections are split over several CTAs
-// (split-KV) and merged by LSE in a second kernel.
+// The selected latent rows of a 64-key tile (all nine 64-dim chunks, 72 KB) are gathered
+// through the block table in one go by two warps with cp.async (16-byte pieces, manual
+// 128-byte swizzle, zeros for empty slots) into one of two tile buffers; the query streams
+// in as 64-dim chunks (TMA, box 128 x 64) through a 3-slot ring.  The same tile feeds the
+// score MMA (K-major B) and P.V (the value chunks as an MN-major B, one 64-dim atom per
+// MMA).  P enters as two bf16 parts hi + lo (the A operand from shared memory), so the
+// probabilities keep ~16 significant bits.  Rescaling of O is lazy: the running max used
+// for P only moves when it grows by more than 2^8.  Long selections are split over several
+// CTAs (split-KV) and merged by LSE in a second kernel.
 //
 //   warps 0..3  softmax: online softmax, P, O rescale, output (one head row per thread)
 //   warp 4      one thread issues tcgen05.mma for S and for P.V, and the commits
-//   warps 5..7  producers: query-chunk TMA, row gathers into the ring and value buffer
+//   warps 5..6  gatherers: each 64-key tile's selected rows, all 9 chunks, by cp.async
+//   warp 7      one thread streams the query's 64-dim chunks by TMA through a 3-slot ring
 #include <cudaTypedefs.h>
 
 #include "dsa_common.cuh"
@@ -34,15 +35,15 @@ namespace dsa {
 
 namespace attn {
 constexpr int kBN = 64;                    // keys per tile
-constexpr int kRing = 3;                   // (query chunk, key chunk) slots, one per producer
+constexpr int kMaxChunks = 9;              // 64-dim chunks of a latent row (576 / 64)
 constexpr int kQChunk = 128 * 128;         // 128 heads x 64 bf16
 constexpr int kKVChunk = kBN * 128;        // 64 keys x 64 bf16
-constexpr int kSlot = kQChunk + kKVChunk;  // 24 KB
+constexpr int kTile = kMaxChunks * kKVChunk;  // one gathered tile, chunk-major: 72 KB
+constexpr int kQRing = 3;                  // query-chunk slots
 constexpr int kMaxVC = 4;                  // 64-dim value chunks per CTA
-constexpr int kVBuf = kMaxVC * kKVChunk;
-constexpr int kOffRing = 0;
-constexpr int kOffV = kOffRing + kRing * kSlot;
-constexpr int kOffP = kOffV + 2 * kVBuf;      // P_hi, then P_lo (bf16, 128 x 64 each)
+constexpr int kOffTile = 0;                // [2] tiles
+constexpr int kOffQ = kOffTile + 2 * kTile;
+constexpr int kOffP = kOffQ + kQRing * kQChunk;  // P_hi, then P_lo (bf16, 128 x 64 each)
 constexpr int kPBytes = 128 * 128;
 constexpr int kOffBar = kOffP + 2 * kPBytes;
 constexpr int kNumBars = 24;
@@ -52,7 +53,11 @@ constexpr int kSmemAlloc = kSmem + 1024;
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-static_assert(kSlot % 1024 == 0 && kVBuf % 1024 == 0, "swizzle atoms");
+constexpr int kProducers = 2;                    // gathering warps 5..6
+constexpr int kThreads = (6 + kProducers) * 32;  // + the query-chunk warp 7: 8 warps, since
+                                                 // registers are granted per 4 warps
+static_assert(kTile % 1024 == 0 && kQChunk % 1024 == 0, "swizzle atoms");
+static_assert(kSmemAlloc <= 232448, "shared memory");
 }  // namespace attn
 
 struct AttnArgs {
@@ -76,7 +81,7 @@ struct AttnArgs {
   float* lse;
   float* part_o;    // [T, splits, H, d_v] fp32 (splits > 1)
   float* part_lse;  // [T, splits, H]
-  int inject;       // test hook: CTA (0, 0) skips its first ring arrival
+  int inject;       // test hook: CTA (0, 0) skips its first query-chunk arrival
 };
 
 // Physical cache row of selected entry v of token t, or -1 if v is empty or invalid.
@@ -95,29 +100,26 @@ __device__ __forceinline__ int resolve_row(int v, int pos, int seq, const AttnAr
   return p * kPage + v % kPage;
 }
 
-constexpr int kProducers = 3;  // producer warps 5..7
-constexpr int kAttnThreads = (5 + kProducers) * 32;
-
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(attn::kThreads, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap, const AttnArgs a) {
   using namespace attn;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* ring_full = bars;             // [kRing]
-  uint64_t* ring_empty = bars + kRing;    // [kRing]
-  uint64_t* v_full = bars + 2 * kRing;    // [2]
-  uint64_t* v_empty = v_full + 2;         // [2]
-  uint64_t* s_full = v_empty + 2;         // [2]
-  uint64_t* s_free = s_full + 2;          // [2]
+  uint64_t* tile_full = bars;           // [2] gathered tile landed (96 producer lanes)
+  uint64_t* tile_empty = bars + 2;      // [2] P.V of that tile done (MMA commit)
+  uint64_t* q_full = bars + 4;          // [kQRing] query chunk landed (TMA)
+  uint64_t* q_empty = q_full + kQRing;  // [kQRing] score MMA done with it (MMA commit)
+  uint64_t* s_full = q_empty + kQRing;  // [2]
+  uint64_t* s_free = s_full + 2;        // [2]
   uint64_t* p_full = s_free + 2;
   uint64_t* pv_done = p_full + 1;
   uint64_t* drain = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
-  uint8_t* ring = smem + kOffRing;
-  uint8_t* vbuf = smem + kOffV;
+  uint8_t* tiles = smem + kOffTile;
+  uint8_t* qring = smem + kOffQ;
   uint8_t* ps = smem + kOffP;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -133,15 +135,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int n_tiles = k1 > k0 ? (k1 - k0 + kBN - 1) / kBN : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kRing; ++i) {
-      mbar_init(&ring_full[i], 1 + 32);  // the query TMA's expect_tx + the 32 gathering lanes
-      mbar_init(&ring_empty[i], 1);
-    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&v_full[i], kProducers * 32);
-      mbar_init(&v_empty[i], 1);
+      mbar_init(&tile_full[i], kProducers * 32);
+      mbar_init(&tile_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
+    }
+    for (int i = 0; i < kQRing; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
     }
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
@@ -159,107 +161,74 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tmem_o = tmem + 2 * kBN;
 
-  if (warp >= 5) {
-    // ---------------------------------------------------------------- producers
-    const int pw = warp - 5;  // owns ring slot pw and every kProducers-th piece of a V tile
-    if (lane == 0) prefetch_tmap(&qmap);
-    int ring_n = 0, q_issued = 0, last_slot_n = -1;
+  if (warp >= 5 && warp < 5 + kProducers) {
+    // ---------------------------------------------------------------- gatherers (2 warps)
+    // Each tile: 64 selected rows x nc chunks x 8 pieces of 16 B, all issued with cp.async
+    // in one go by the 64 lanes, then one wait for the whole tile.
+    const int pl = threadIdx.x - 5 * 32;  // 0..63
     bool ok = true;
     for (int i = 0; ok && i < n_tiles; ++i) {
-      // physical rows of the tile's 64 slots: lane l resolves slots l and l + 32
+      const int b = i & 1;
+      if (!mbar_wait_warp(&tile_empty[b], ((i >> 1) & 1) ^ 1, abort_flag, 42)) break;
       int rows[2];
       for (int u = 0; u < 2; ++u) {
         const int slot = k0 + i * kBN + lane + 32 * u;
         const int v = slot < k1 ? a.idx[static_cast<size_t>(t) * a.k + slot] : -1;
-        rows[u] = resolve_row(v, pos, seq, a, pw == 0);
+        rows[u] = resolve_row(v, pos, seq, a, warp == 5);
       }
-      // score operands: chunk c goes to ring slot n % kRing, filled by warp n % kRing
-      for (int c = 0; c < nc; ++c, ++ring_n) {
-        if (ring_n % kRing != pw) continue;
-        if (!mbar_wait_warp(&ring_empty[pw], ((ring_n / kRing) & 1) ^ 1, abort_flag, 41)) {
-          ok = false;
-          break;
-        }
-        uint8_t* sb = ring + pw * kSlot;
-        if (lane == 0 && !(a.inject && blockIdx.x == 0 && blockIdx.y == 0 && ring_n == 0)) {
-          mbar_arrive_expect_tx(&ring_full[pw], kQChunk);
-          tma_load_2d(sb, &qmap, &ring_full[pw], c * 64, t * a.H);
-          ++q_issued;
-        }
-        last_slot_n = ring_n;
-        // 64 rows x 8 pieces of 16 B: lane handles pieces lane + 32 j, 8 loads in flight
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint4 v[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int p = lane + 32 * (8 * half + j), r = p >> 3, c16 = p & 7;
-            const int r0 = __shfl_sync(0xffffffffu, rows[0], r & 31);
-            const int r1 = __shfl_sync(0xffffffffu, rows[1], r & 31);
-            const int row = (r >> 5) ? r1 : r0;
-            const int d0 = c * 64 + c16 * 8;
-            v[j] = (row >= 0 && d0 < a.d_kv) ? *reinterpret_cast<const uint4*>(
-                                                   a.kv + static_cast<size_t>(row) * a.d_kv + d0)
-                                             : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int p = lane + 32 * (8 * half + j), r = p >> 3, c16 = p & 7;
-            *reinterpret_cast<uint4*>(sb + kQChunk + swz_offset(r, c16 * 16, 128)) = v[j];
-          }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&ring_full[pw]);
+      uint8_t* tb = tiles + b * kTile;
+      const int pieces = kBN * 8 * nc;  // (row, chunk, 16-byte piece)
+      for (int p = pl; p < pieces; p += kProducers * 32) {
+        const int c = p / (kBN * 8), rem = p % (kBN * 8), r = rem >> 3, c16 = rem & 7;
+        // the physical row of tile row r sits in lane r % 32 (slot r < 32: rows[0], else rows[1])
+        const int r0 = __shfl_sync(0xffffffffu, rows[0], r & 31);
+        const int r1 = __shfl_sync(0xffffffffu, rows[1], r & 31);
+        const int row = (r >> 5) ? r1 : r0;
+        const int d0 = c * 64 + c16 * 8;
+        const int valid = row >= 0 ? max(0, min(8, a.d_kv - d0)) : 0;
+        const uint16_t* src = valid ? a.kv + static_cast<size_t>(row) * a.d_kv + d0 : a.kv;
+        cp_async_16(tb + c * kKVChunk + swz_offset(r, c16 * 16, 128), src, valid * 2);
       }
-      if (!ok) break;
-      // this warp's share of the value tile: pieces lane + 32 j with j % kProducers == pw
-      const int vb = i & 1;
-      if (!mbar_wait_warp(&v_empty[vb], ((i >> 1) & 1) ^ 1, abort_flag, 42)) break;
-      for (int vc = 0; vc < a.nvg; ++vc) {
-        uint4 v[6];
-#pragma unroll
-        for (int jj = 0; jj < 6; ++jj) {
-          const int j = pw + kProducers * jj;
-          if (j >= 16) break;
-          const int p = lane + 32 * j, r = p >> 3, c16 = p & 7;
-          const int r0 = __shfl_sync(0xffffffffu, rows[0], r & 31);
-          const int r1 = __shfl_sync(0xffffffffu, rows[1], r & 31);
-          const int row = (r >> 5) ? r1 : r0;
-          const int d0 = (vc0 + vc) * 64 + c16 * 8;
-          v[jj] = row >= 0 ? *reinterpret_cast<const uint4*>(a.kv + static_cast<size_t>(row) *
-                                                                         a.d_kv + d0)
-                           : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int jj = 0; jj < 6; ++jj) {
-          const int j = pw + kProducers * jj;
-          if (j >= 16) break;
-          const int p = lane + 32 * j, r = p >> 3, c16 = p & 7;
-          *reinterpret_cast<uint4*>(vbuf + vb * kVBuf + vc * kKVChunk +
-                                    swz_offset(r, c16 * 16, 128)) = v[jj];
-        }
-      }
+      cp_async_commit();
+      cp_async_wait<0>();
       fence_proxy_async_smem();
-      mbar_arrive(&v_full[vb]);
+      mbar_arrive(&tile_full[b]);
     }
-    // the last query TMA of this warp's slot must land before the CTA exits
-    if (lane == 0 && q_issued > 0 && last_slot_n >= 0)
-      mbar_wait_drain(&ring_full[pw], (last_slot_n / kRing) & 1);
+    cp_async_wait<0>();
+  } else if (warp == 5 + kProducers) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- query-chunk TMA
+      prefetch_tmap(&qmap);
+      int qn = 0;
+      for (int i = 0; i < n_tiles; ++i)
+        for (int c = 0; c < nc; ++c, ++qn) {
+          const int slot = qn % kQRing;
+          if (!mbar_wait(&q_empty[slot], ((qn / kQRing) & 1) ^ 1, abort_flag, 41)) {
+            i = n_tiles;
+            break;
+          }
+          if (a.inject && blockIdx.x == 0 && blockIdx.y == 0 && qn == 0) continue;
+          mbar_arrive_expect_tx(&q_full[slot], kQChunk);
+          tma_load_2d(qring + slot * kQChunk, &qmap, &q_full[slot], c * 64, t * a.H);
+        }
+      // every issued copy must land before the CTA exits
+      for (int m = max(0, qn - kQRing); m < qn; ++m)
+        mbar_wait_drain(&q_full[m % kQRing], (m / kQRing) & 1);
+    }
     __syncwarp();
   } else if (warp == 4) {
-    // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
       const uint32_t idesc_s = instr_desc(128, kBN, 1, 1, 0, 0);
       const uint32_t idesc_pv = instr_desc(128, 64, 1, 1, 0, 1);
-      const uint32_t ring_base = smem_u32(ring), v_base = smem_u32(vbuf), p_base = smem_u32(ps);
+      const uint32_t tile_base = smem_u32(tiles), q_base = smem_u32(qring), p_base = smem_u32(ps);
       bool ok = true;
-      int ring_n = 0;
+      int qn = 0;
       auto do_pv = [&](int j) -> bool {
         if (!mbar_wait(p_full, j & 1, abort_flag, 45)) return false;
-        if (!mbar_wait(&v_full[j & 1], (j >> 1) & 1, abort_flag, 46)) return false;
         tc_fence_after();
         fence_proxy_async_smem();
-        const uint32_t vb = v_base + (j & 1) * kVBuf;
+        const uint32_t tb = tile_base + (j & 1) * kTile;
         // P = P_hi + P_lo (both bf16): the second product restores the bits a single
         // bf16 P would lose, so the value weights are exact to ~2^-17
         for (int vc = 0; vc < a.nvg; ++vc)
@@ -269,30 +238,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int part = 0; part < 2; ++part)
               mma_bf16(tmem_o + vc * 64,
                        smem_desc(p_base + part * kPBytes + ks * 32, 16, 1024, kSw128),
-                       smem_desc(vb + vc * kKVChunk + ks * 2048, kKVChunk, 1024, kSw128),
+                       smem_desc(tb + (vc0 + vc) * kKVChunk + ks * 2048, kKVChunk, 1024, kSw128),
                        idesc_pv, (j > 0 || ks > 0 || part > 0) ? 1u : 0u);
-        mma_commit(&v_empty[j & 1]);
+        mma_commit(&tile_empty[j & 1]);
         mma_commit(pv_done);
         return true;
       };
       for (int i = 0; ok && i < n_tiles; ++i) {
         const int st = i & 1;
         if (!mbar_wait(&s_free[st], ((i >> 1) & 1) ^ 1, abort_flag, 43)) break;
-        for (int c = 0; c < nc; ++c) {
-          const int slot = ring_n % kRing;
-          if (!mbar_wait(&ring_full[slot], (ring_n / kRing) & 1, abort_flag, 44)) {
+        if (!mbar_wait(&tile_full[st], (i >> 1) & 1, abort_flag, 46)) break;
+        const uint32_t tb = tile_base + st * kTile;
+        for (int c = 0; c < nc; ++c, ++qn) {
+          const int slot = qn % kQRing;
+          if (!mbar_wait(&q_full[slot], (qn / kQRing) & 1, abort_flag, 44)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sb = ring_base + slot * kSlot;
+          fence_proxy_async_smem();
+          const uint32_t qb = q_base + slot * kQChunk;
           const int w = min(64, a.d_kv - c * 64);
           for (int ks = 0; ks < (w + 15) / 16; ++ks)
-            mma_bf16(tmem + st * kBN, smem_desc(sb + ks * 32, 16, 1024, kSw128),
-                     smem_desc(sb + kQChunk + ks * 32, 16, 1024, kSw128), idesc_s,
+            mma_bf16(tmem + st * kBN, smem_desc(qb + ks * 32, 16, 1024, kSw128),
+                     smem_desc(tb + c * kKVChunk + ks * 32, 16, 1024, kSw128), idesc_s,
                      (c > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(&ring_empty[slot]);
-          ++ring_n;
+          mma_commit(&q_empty[slot]);
         }
         if (!ok) break;
         mma_commit(&s_full[st]);
@@ -482,16 +453,25 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restri
   }
   __syncthreads();
   for (int d = threadIdx.x * 4; d < d_v; d += blockDim.x * 4) {
+    // every split's partial is loaded before the sum (independent loads, one round trip)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < splits; ++s) {
-      const float w = wsh[s];
-      if (w == 0.f) continue;
-      const float4 v = *reinterpret_cast<const float4*>(
-          part_o + ((static_cast<size_t>(t) * splits + s) * H + h) * d_v + d);
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
+    constexpr int kBatch = 16;
+    for (int s0 = 0; s0 < splits; s0 += kBatch) {
+      float4 v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        v[u] = s0 + u < splits ? *reinterpret_cast<const float4*>(
+                                     part_o + ((static_cast<size_t>(t) * splits + s0 + u) * H + h) *
+                                                  d_v + d)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const float w = s0 + u < splits ? wsh[s0 + u] : 0.f;
+        acc.x = fmaf(w, v[u].x, acc.x);
+        acc.y = fmaf(w, v[u].y, acc.y);
+        acc.z = fmaf(w, v[u].z, acc.z);
+        acc.w = fmaf(w, v[u].w, acc.w);
+      }
     }
     uint2 pk = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
     *reinterpret_cast<uint2*>(out + (static_cast<size_t>(t) * H + h) * d_v + d) = pk;
@@ -597,7 +577,7 @@ cudaError_t launch_attn(const AttnLaunch& L) {
     a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(L.ws) +
                                           ((o + 255) & ~static_cast<size_t>(255)));
   }
-  sparse_mla_kernel<<<dim3(groups * splits, T), kAttnThreads, attn::kSmemAlloc, L.stream>>>(qmap,
+  sparse_mla_kernel<<<dim3(groups * splits, T), attn::kThreads, attn::kSmemAlloc, L.stream>>>(qmap,
                                                                                            a);
   count_launch();
   cudaError_t e = cudaGetLastError();

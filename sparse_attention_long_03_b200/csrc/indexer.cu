@@ -96,22 +96,23 @@ __global__ void __launch_bounds__(1024) indexer_prep_kernel(const int32_t* __res
                                                             int32_t T, int32_t batch,
                                                             int32_t max_pos, int32_t pos_cap,
                                                             void* ws, uint32_t* zero,
-                                                            int64_t zero_words) {
+                                                            int64_t zero_words, int run_tokens) {
   __shared__ int sm[33];
   pdl_wait();
   pdl_trigger();
   for (int64_t i = threadIdx.x; i < zero_words; i += blockDim.x) zero[i] = 0u;
   PlanView v = plan_view(ws, T);
-  const int n_groups = (T + kRunTokens - 1) / kRunTokens;
+  const int G = run_tokens;  // 1 (decode) or kRunTokens
+  const int n_groups = (T + G - 1) / G;
   int carry = 0;
   for (int base = 0; base < n_groups; base += blockDim.x) {
     const int g = base + threadIdx.x;
     int nr = 0, cnt = 0, seqs[kRunTokens], poss[kRunTokens];
     bool ok[kRunTokens], uniform = true;
     if (g < n_groups) {
-      cnt = min(kRunTokens, T - kRunTokens * g);
+      cnt = min(G, T - G * g);
       for (int j = 0; j < cnt; ++j) {
-        const int t = kRunTokens * g + j;
+        const int t = G * g + j;
         seqs[j] = tok_seq[t];
         poss[j] = tok_pos[t];
         ok[j] = seqs[j] >= 0 && seqs[j] < batch && poss[j] >= 0 && poss[j] <= max_pos &&
@@ -130,13 +131,13 @@ __global__ void __launch_bounds__(1024) indexer_prep_kernel(const int32_t* __res
       if (uniform) {
         int mp = poss[0];
         for (int j = 1; j < cnt; ++j) mp = max(mp, poss[j]);
-        v.tok0[off] = kRunTokens * g;
+        v.tok0[off] = G * g;
         v.ntok[off] = cnt;
         v.seq[off] = seqs[0];
         v.maxpos[off] = mp;
       } else {
         for (int j = 0; j < cnt; ++j) {
-          v.tok0[off + j] = kRunTokens * g + j;
+          v.tok0[off + j] = G * g + j;
           v.ntok[off + j] = 1;
           v.seq[off + j] = ok[j] ? seqs[j] : 0;
           v.maxpos[off + j] = ok[j] ? poss[j] : -1;  // no work for an invalid token
@@ -188,22 +189,25 @@ __host__ __device__ constexpr int pow2ceil(int x) {
   return p;
 }
 
-template <int DI, int HP>
+template <int DI, int HP, int RT>
 struct IdxCfg {
   static constexpr int kStages = DI == 128 ? 6 : 8;
   static constexpr int kTileBytes = kKeyTile * DI;
-  static constexpr int kQBytes = kRunTokens * HP * DI;
-  static constexpr int kNC = kRunTokens * HP;  // TMEM columns of one accumulator buffer
-  static constexpr int kTmemCols = pow2ceil(2 * kNC);
+  static constexpr int kQBytes = (RT * HP * DI + 1023) / 1024 * 1024;  // whole swizzle atoms
+  static constexpr int kNC = RT * HP;  // TMEM columns of one accumulator buffer
+  // accumulator buffers: as many as fit TMEM (up to 8), so the MMA can run that many
+  // key tiles ahead of the epilogue
+  static constexpr int kNBuf = (512 / kNC) < 8 ? (512 / kNC) : 8;
+  static constexpr int kTmemCols = pow2ceil(kNBuf * kNC);
   static constexpr int kOffK = 0;
   static constexpr int kOffQ = kOffK + kStages * kTileBytes;
   static constexpr int kOffWq = kOffQ + 2 * kQBytes;
-  static constexpr int kOffMeta = kOffWq + 2 * kRunTokens * HP * 4;
-  static constexpr int kOffScale = kOffMeta + 64;                 // [S][128] fp32
+  static constexpr int kOffMeta = kOffWq + 2 * kRunTokens * HP * 4;  // qpos, qtok, qn [2][4]
+  static constexpr int kOffScale = kOffMeta + 128;                // [S][128] fp32
   static constexpr int kOffPage = kOffScale + kStages * kKeyTile * 4;  // [S][2] int32
   static constexpr int kOffHist = kOffPage + kStages * 8 + 64;
   static constexpr int kOffBar = kOffHist + kRunTokens * 2048 * 4;
-  static constexpr int kNumBars = 2 * kStages + 11;
+  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kNBuf + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16;
   static constexpr int kSmemAlloc = kSmem + 1024;
@@ -231,10 +235,11 @@ struct ItemWalker {
   __device__ void advance() { ++i; }
 };
 
-template <int DI, int HP>
+template <int DI, int HP, int RT>
 __global__ void __launch_bounds__(192, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap kmap, const IdxArgs a) {
-  using C = IdxCfg<DI, HP>;
+  using C = IdxCfg<DI, HP, RT>;
+  constexpr int NB = C::kNBuf;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -244,14 +249,15 @@ __global__ void __launch_bounds__(192, 1)
   float* wq = reinterpret_cast<float*>(smem + C::kOffWq);
   int* qpos = reinterpret_cast<int*>(smem + C::kOffMeta);
   int* qtok = qpos + 2 * kRunTokens;
+  int* qn = qtok + 2 * kRunTokens;  // tokens in the run held by each Q slot
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* qfull = bars + 2 * S;
   uint64_t* qempty = qfull + 2;
-  uint64_t* tfull = qempty + 2;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* tfull = qempty + 2;   // [NB]
+  uint64_t* tempty = tfull + NB;  // [NB]
+  uint64_t* drain = tempty + NB;
   uint64_t* hist_full = drain + 1;
   uint64_t* hist_free = drain + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -269,8 +275,10 @@ __global__ void __launch_bounds__(192, 1)
     for (int q = 0; q < 2; ++q) {
       mbar_init(&qfull[q], 1);
       mbar_init(&qempty[q], 1 + 4);
-      mbar_init(&tfull[q], 1);
-      mbar_init(&tempty[q], 4);
+    }
+    for (int b = 0; b < NB; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
     }
     mbar_init(drain, 1);
     mbar_init(hist_full, 4);
@@ -339,6 +347,7 @@ __global__ void __launch_bounds__(192, 1)
           qpos[slot * kRunTokens + lane] = a.tok_pos[tok0 + lane];
           qtok[slot * kRunTokens + lane] = tok0 + lane;
         }
+        if (lane == 0) qn[slot] = ntok;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&qfull[slot]);
@@ -394,8 +403,8 @@ __global__ void __launch_bounds__(192, 1)
           slot = wk.rc & 1;
           if (!mbar_wait(&qfull[slot], (wk.rc >> 1) & 1, abort_flag, 13)) break;
         }
-        const int ab = n & 1;
-        if (!mbar_wait(&tempty[ab], ((n >> 1) & 1) ^ 1, abort_flag, 14)) break;
+        const int ab = n % NB;
+        if (!mbar_wait(&tempty[ab], ((n / NB) & 1) ^ 1, abort_flag, 14)) break;
         const int stage = n % S;
         if (!mbar_wait(&full[stage], (n / S) & 1, abort_flag, 15)) break;
         tc_fence_after();
@@ -420,24 +429,28 @@ __global__ void __launch_bounds__(192, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     int n = 0, n_flush = 0;
-    int slot = 0;
+    int slot = 0, ntok = 0;
+    float wreg[RT == 1 ? HP : 1];  // head weights of a one-token run, kept in registers
     for (; wk.next(); wk.advance(), ++n) {
-      const int r = wk.r;
       if (wk.new_run) {
         slot = wk.rc & 1;
         if (!mbar_wait_warp(&qfull[slot], (wk.rc >> 1) & 1, abort_flag, 16)) break;
+        ntok = qn[slot];
+        if constexpr (RT == 1) {
+#pragma unroll
+          for (int h = 0; h < HP; ++h) wreg[h] = wq[slot * kRunTokens * HP + h];
+        }
       }
-      const int ab = n & 1;
-      if (!mbar_wait_warp(&tfull[ab], (n >> 1) & 1, abort_flag, 17)) break;
+      const int ab = n % NB;
+      if (!mbar_wait_warp(&tfull[ab], (n / NB) & 1, abort_flag, 17)) break;
       tc_fence_after();
       const int s = wk.tile * kKeyTile + row;
-      const int ntok = pv.ntok[r];
       const int stage = n % S;
       // the stage's scales and page ids (complete: the MMA already waited for it)
       if (!mbar_wait_warp(&full[stage], (n / S) & 1, abort_flag, 18)) break;
       const float ks = pages[stage * 2 + (row >> 6)] >= 0 ? scales[stage * kKeyTile + row]
                                                            : __int_as_float(0x7fc00000);
-      for (int j = 0; j < ntok; ++j) {
+      for (int j = 0; j < (RT == 1 ? 1 : ntok); ++j) {
         float x[HP];
         const uint32_t taddr =
             tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::kNC + j * HP;
@@ -449,12 +462,20 @@ __global__ void __launch_bounds__(192, 1)
         }
         tmem_wait_ld();
         if (s <= qpos[slot * kRunTokens + j]) {
-          const float* wv = wq + (slot * kRunTokens + j) * HP;
           float acc0 = 0.f, acc1 = 0.f;
+          if constexpr (RT == 1) {
 #pragma unroll
-          for (int h = 0; h < HP; h += 2) {
-            acc0 = fmaf(fmaxf(x[h], 0.f), wv[h], acc0);
-            acc1 = fmaf(fmaxf(x[h + 1], 0.f), wv[h + 1], acc1);
+            for (int h = 0; h < HP; h += 2) {
+              acc0 = fmaf(fmaxf(x[h], 0.f), wreg[h], acc0);
+              acc1 = fmaf(fmaxf(x[h + 1], 0.f), wreg[h + 1], acc1);
+            }
+          } else {
+            const float* wv = wq + (slot * kRunTokens + j) * HP;
+#pragma unroll
+            for (int h = 0; h < HP; h += 2) {
+              acc0 = fmaf(fmaxf(x[h], 0.f), wv[h], acc0);
+              acc1 = fmaf(fmaxf(x[h + 1], 0.f), wv[h + 1], acc1);
+            }
           }
           const float v = (acc0 + acc1) * ks;
           a.logits[static_cast<int64_t>(qtok[slot * kRunTokens + j]) * a.ld + s] = v;
@@ -515,14 +536,14 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-template <int DI, int HP>
+template <int DI, int HP, int RT>
 static cudaError_t launch_indexer_t(const IndexerLaunch& L, const CUtensorMap& map, int grid) {
-  using C = IdxCfg<DI, HP>;
+  using C = IdxCfg<DI, HP, RT>;
   static int attr_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_dev != dev) {
-    cudaError_t e = cudaFuncSetAttribute(indexer_kernel<DI, HP>,
+    cudaError_t e = cudaFuncSetAttribute(indexer_kernel<DI, HP, RT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemAlloc);
     if (e != cudaSuccess) return e;
@@ -544,8 +565,8 @@ static cudaError_t launch_indexer_t(const IndexerLaunch& L, const CUtensorMap& m
   a.T = L.queries->n_tokens;
   a.hist = L.hist;
   a.inject = take_injection(1);
-  return launch_pdl(indexer_kernel<DI, HP>, dim3(grid), dim3(192), C::kSmemAlloc, L.stream, map,
-                    a);
+  return launch_pdl(indexer_kernel<DI, HP, RT>, dim3(grid), dim3(192), C::kSmemAlloc, L.stream,
+                    map, a);
 }
 
 cudaError_t launch_indexer(const IndexerLaunch& L) {
@@ -553,9 +574,12 @@ cudaError_t launch_indexer(const IndexerLaunch& L) {
   const dsa_queries* q = L.queries;
   const int T = q->n_tokens;
   if (T == 0) return cudaSuccess;
+  // one query token per sequence on average (decode): runs of one token, which lets the
+  // kernel keep eight accumulator buffers in TMEM; otherwise runs of up to four tokens
+  const int RT = T <= c->batch ? 1 : kRunTokens;
   cudaError_t e = launch_pdl(indexer_prep_kernel, dim3(1), dim3(1024), 0, L.stream, q->tok_seq,
                              q->tok_pos, T, c->batch, q->max_pos, c->max_blocks_per_seq * kPage,
-                             L.ws, L.zero, L.zero_words);
+                             L.ws, L.zero, L.zero_words, RT);
   if (e != cudaSuccess) return e;
 
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
@@ -579,8 +603,10 @@ cudaError_t launch_indexer(const IndexerLaunch& L) {
   const int grid = static_cast<int>(tiles_ub < num_sms() ? tiles_ub : num_sms());
   if (grid <= 0) return cudaSuccess;
   const int HP = L.n_idx_heads <= 16 ? 16 : (L.n_idx_heads <= 32 ? 32 : 64);
-#define DSA_IDX_CASE(di, hp) \
-  if (DI == di && HP == hp) return launch_indexer_t<di, hp>(L, map, grid);
+#define DSA_IDX_CASE(di, hp)                                             \
+  if (DI == di && HP == hp)                                              \
+    return RT == 1 ? launch_indexer_t<di, hp, 1>(L, map, grid)           \
+                   : launch_indexer_t<di, hp, kRunTokens>(L, map, grid);
   DSA_IDX_CASE(128, 64)
   DSA_IDX_CASE(128, 32)
   DSA_IDX_CASE(128, 16)

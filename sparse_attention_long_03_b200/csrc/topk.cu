@@ -55,6 +55,12 @@ struct CandGlobal {
   __device__ uint32_t key(int i) const { return float_to_ordered(row[list[i]]); }
   __device__ int index(int i) const { return list[i]; }
 };
+struct RowCachedOff {
+  const uint32_t* keys;
+  int off;
+  __device__ uint32_t key(int i) const { return keys[i]; }
+  __device__ int index(int i) const { return off + i; }
+};
 struct RowCached {
   const uint32_t* keys;
   __device__ uint32_t key(int i) const { return keys[i]; }
@@ -373,8 +379,12 @@ __global__ void __launch_bounds__(kTopkDecThreads, 1)
   const int c1 = static_cast<int>(static_cast<int64_t>(n) * (c + 1) / chunks);
   int32_t* sa = ws.scr_a + static_cast<int64_t>(t) * ld;
   int32_t* sb = ws.scr_b + static_cast<int64_t>(t) * ld;
+  // this CTA's chunk, read once into shared memory with every load in flight
+  uint32_t* ck = reinterpret_cast<uint32_t*>(topk_smem_raw + kTopkSmemBase);
+  for (int i = threadIdx.x; i < c1 - c0; i += blockDim.x) ck[i] = float_to_ordered(row[c0 + i]);
+  __syncthreads();
   const int2 cnt = ordered_pass(
-      sm, RowGlobalOff{row, c0}, c1 - c0,
+      sm, RowCachedOff{ck, c0}, c1 - c0,
       [b1](uint32_t key) { return (key >> 21) > b1 ? 1 : ((key >> 21) == b1 ? 2 : 0); }, sa, c0,
       [sb, c0](int r, uint32_t, int i) { sb[c0 + r] = i; }, c1 - c0);
   if (threadIdx.x == 0) {
@@ -455,8 +465,16 @@ size_t topk_decode_ws_bytes(int32_t T, int64_t ld, int chunks) {
          al(static_cast<size_t>(T) * chunks * 8) + 2 * al(static_cast<size_t>(T) * ld * 4);
 }
 
+// Largest chunk a CTA of the decode kernel reads (rows are at most max_pos + 1 long).
+static size_t decode_chunk_cap(int32_t max_pos, int chunks) {
+  return (static_cast<size_t>(max_pos) + 1 + chunks - 1) / chunks + 1;
+}
+
 int topk_decode_chunks(int32_t T, int32_t max_pos) {
   int c = T > 0 ? num_sms() / T : 1;
+  // a chunk must fit the shared-memory row cache
+  const int min_c = static_cast<int>((static_cast<size_t>(max_pos) + kTopkRowCache) / kTopkRowCache);
+  if (c < min_c) c = min_c;
   const int by_len = (max_pos + 1) / 1024 + 1;
   if (c > by_len) c = by_len;
   if (c > kTopkMaxChunks) c = kTopkMaxChunks;
@@ -490,13 +508,16 @@ cudaError_t launch_topk_decode(const float* logits, int64_t ld, const dsa_querie
   if (attr_dev != dev) {
     cudaError_t e = cudaFuncSetAttribute(topk_decode_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kTopkSmemBase));
+                                         static_cast<int>(kTopkSmemMax));
     if (e != cudaSuccess) return e;
     attr_dev = dev;
   }
   TopkDecodeWs w{L.hist, L.arrive, L.counts, L.scr_a, L.scr_b};
-  return launch_pdl(topk_decode_kernel, dim3(chunks, q->n_tokens), dim3(kTopkDecThreads),
-                    kTopkSmemBase, stream, logits, ld, q->tok_pos, q->max_pos, k, idx, w, chunks);
+  const size_t cap = decode_chunk_cap(q->max_pos, chunks);
+  if (cap > static_cast<size_t>(kTopkRowCache)) return cudaErrorNotSupported;
+  const size_t smem = kTopkSmemBase + cap * sizeof(uint32_t);
+  return launch_pdl(topk_decode_kernel, dim3(chunks, q->n_tokens), dim3(kTopkDecThreads), smem,
+                    stream, logits, ld, q->tok_pos, q->max_pos, k, idx, w, chunks);
 }
 
 }  // namespace dsa

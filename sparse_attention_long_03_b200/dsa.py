@@ -29,14 +29,17 @@ EXPORTED = ("dsa_indexer_logits", "dsa_indexer_workspace_size", "dsa_indexer_log
             "dsa_topk_workspace_size", "dsa_sparse_mla_attn", "dsa_attn_workspace_size",
             "dsa_forward", "dsa_forward_workspace_size", "dsa_read_device_status",
             "dsa_launch_count", "dsa_status_string", "dsa_abi_version", "dsa_debug_inject",
-            "dsa_debug_timeout_site")
+            "dsa_debug_timeout_site", "dsa_last_cuda_error")
 
 
 class DsaError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
+        extra = ""
+        if status == 4:
+            extra = f" (cudaError_t {lib().dsa_last_cuda_error()})"
         super().__init__(f"{fn} -> {STATUS_NAMES.get(status, status)}: "
-                         f"{lib().dsa_status_string(status).decode()}")
+                         f"{lib().dsa_status_string(status).decode()}{extra}")
 
 
 class PagedCache(ctypes.Structure):
@@ -89,6 +92,7 @@ def lib() -> ctypes.CDLL:
             "dsa_abi_version": (I32, []),
             "dsa_debug_inject": (I32, [I32]),
             "dsa_debug_timeout_site": (ctypes.c_uint32, []),
+            "dsa_last_cuda_error": (I32, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
