@@ -366,8 +366,13 @@ def run_ours(args, rank, world, local):
         st_topk(0)
     stream.synchronize()
     reps = max(50, min(args.steps, 2000))
-    stages = {"indexer_us": time_stage(st_indexer, reps), "topk_us": time_stage(st_topk, reps),
-              "attention_us": time_stage(st_attn, reps)}
+    # indexer_us: prep + indexer kernels (dsa_indexer_logits); attention_us: attention +
+    # split combine (dsa_sparse_mla_attn); topk_rowwise_us: the one-CTA-per-row top-k of
+    # dsa_topk, which the decode forward replaces by its multi-CTA top-k fed by the
+    # indexer's histogram
+    stages = {"indexer_us": time_stage(st_indexer, reps),
+              "attention_us": time_stage(st_attn, reps),
+              "topk_rowwise_us": time_stage(st_topk, reps)}
 
     # end to end through the public API with host buffers: per step, H2D of the step's
     # query inputs from pinned memory, the forward, D2H of the output and LSE
@@ -433,13 +438,7 @@ def run_ours(args, rank, world, local):
     idx_us = stages["indexer_us"]
     achieved = bytes_model["indexer"] / (idx_us * 1e-6) / 1e9
     path_gbs = (bytes_model["indexer"] + bytes_model["gather"]) / (ms_per_step * 1e-3) / 1e9
-    traffic = None
-    tr_path = os.path.join(ROOT, "profiles", "indexer_decode_128k_traffic.json")
-    if os.path.exists(tr_path):
-        try:
-            traffic = json.load(open(tr_path)).get("bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = measured_traffic()
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -469,6 +468,25 @@ def run_ours(args, rank, world, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, cache, qs)
     return line
+
+
+def measured_traffic():
+    """DRAM bytes per indexer launch from the committed ncu summary, or None when the
+    kernel source has changed since those counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "indexer_decode_128k.md")
+    src = os.path.join(ROOT, "sparse_attention_long_03_b200", "csrc", "indexer.cu")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for ln in open(path):
+        if ln.startswith("- ") and ":" in ln:
+            k, v = ln[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    have = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if fields.get("indexer.cu sha256") != have or "dram bytes per launch" not in fields:
+        return None
+    return int(fields["dram bytes per launch"].replace(",", ""))
 
 
 def main():

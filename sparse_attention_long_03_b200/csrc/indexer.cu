@@ -13,9 +13,11 @@
 // without any cross-thread traffic.  Keys stream from the paged cache with TMA (one
 // 64-token page per box, swizzled for the MMA), through a multi-stage mbarrier ring.
 //
-//   warp 0      producer: Q rows of each run (manual swizzled stores) + TMA key pages
+//   warp 0      producer: key pages by TMA and their scales by bulk copy, up to eight key
+//               tiles per pass (one page per lane)
 //   warp 1      one thread issues tcgen05.mma (kind::f8f6f4) and tcgen05.commit
-//   warps 2..5  epilogue: tcgen05.ld -> ReLU . w -> logits (coalesced fp32 stores)
+//   warps 2..5  epilogue: tcgen05.ld -> ReLU . w -> logits (coalesced fp32 stores); they
+//               also stage each run's query rows (manual swizzled stores) one run ahead
 //
 // A small planner kernel first groups the query tokens into runs of up to 4 tokens of
 // the same sequence (they share every key tile) and lays the (run, key tile) work items
@@ -101,6 +103,7 @@ __global__ void __launch_bounds__(1024) indexer_prep_kernel(const int32_t* __res
   pdl_wait();
   pdl_trigger();
   for (int64_t i = threadIdx.x; i < zero_words; i += blockDim.x) zero[i] = 0u;
+  if (ws == nullptr) return;  // the indexer plans one-token runs itself
   PlanView v = plan_view(ws, T);
   const int G = run_tokens;  // 1 (decode) or kRunTokens
   const int n_groups = (T + G - 1) / G;
@@ -170,18 +173,27 @@ struct IdxArgs {
   const int32_t* block_table;
   int32_t max_blocks;
   int32_t num_blocks;
+  const int32_t* tok_seq;
   const int32_t* tok_pos;
+  int32_t batch;
+  int32_t max_pos;
+  int32_t pos_cap;
   const uint8_t* q8;
   const float* q_scale;
   const float* w;
   int32_t n_idx_heads;
   float* logits;
   int64_t ld;
-  void* plan;
+  void* plan;  // the prep kernel's plan, or null: the kernel plans one-token runs itself
   int32_t T;
   uint32_t* hist;  // [T][2048] first-digit histogram of the ordered logits, or null
-  int inject;      // test hook: the CTA owning item 0 skips its first stage's arrival
+  int inject;      // test hook: the CTA owning item 0 skips its first stage's arrivals
 };
+
+// Query tokens up to which one-token runs are planned inside the indexer kernel.
+constexpr int kInlinePlanMax = 64;
+// Key tiles the producer warp issues per pass (two pages each, one per lane), at most.
+constexpr int kProducerBatch = 8;
 
 __host__ __device__ constexpr int pow2ceil(int x) {
   int p = 32;
@@ -191,7 +203,9 @@ __host__ __device__ constexpr int pow2ceil(int x) {
 
 template <int DI, int HP, int RT>
 struct IdxCfg {
-  static constexpr int kStages = DI == 128 ? 6 : 8;
+  static constexpr int kStages = RT == 1 ? 10 : (DI == 128 ? 6 : 8);
+  // key tiles per producer pass: distinct stages and scale slots
+  static constexpr int kBatch = kProducerBatch < kStages ? kProducerBatch : kStages;
   static constexpr int kTileBytes = kKeyTile * DI;
   static constexpr int kQBytes = (RT * HP * DI + 1023) / 1024 * 1024;  // whole swizzle atoms
   static constexpr int kNC = RT * HP;  // TMEM columns of one accumulator buffer
@@ -199,20 +213,26 @@ struct IdxCfg {
   // key tiles ahead of the epilogue
   static constexpr int kNBuf = (512 / kNC) < 8 ? (512 / kNC) : 8;
   static constexpr int kTmemCols = pow2ceil(kNBuf * kNC);
+  // scale slots: the epilogue trails the producer by up to kStages + kNBuf tiles
+  static constexpr int kScaleSlots = 16;
+  static_assert(kScaleSlots >= kBatch, "a producer pass needs distinct scale slots");
+  static constexpr int kPlanWords = 4 + 5 * kInlinePlanMax + 1;
   static constexpr int kOffK = 0;
   static constexpr int kOffQ = kOffK + kStages * kTileBytes;
   static constexpr int kOffWq = kOffQ + 2 * kQBytes;
   static constexpr int kOffMeta = kOffWq + 2 * kRunTokens * HP * 4;  // qpos, qtok, qn [2][4]
-  static constexpr int kOffScale = kOffMeta + 128;                // [S][128] fp32
-  static constexpr int kOffPage = kOffScale + kStages * kKeyTile * 4;  // [S][2] int32
-  static constexpr int kOffHist = kOffPage + kStages * 8 + 64;
-  static constexpr int kOffBar = kOffHist + kRunTokens * 2048 * 4;
-  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kNBuf + 3;
+  static constexpr int kOffScale = kOffMeta + 128;                // [kScaleSlots][128] fp32
+  static constexpr int kOffPage = kOffScale + kScaleSlots * kKeyTile * 4;  // [slots][2] int32
+  static constexpr int kOffPlan = kOffPage + kScaleSlots * 8;
+  static constexpr int kOffHist = kOffPlan + (kPlanWords * 4 + 63) / 64 * 64;
+  static constexpr int kOffBar = kOffHist + RT * 2048 * 4;
+  static constexpr int kNumBars = 2 * kStages + 2 * kScaleSlots + 4 + 2 * kNBuf + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16;
   static constexpr int kSmemAlloc = kSmem + 1024;
   static constexpr uint32_t kSwz = DI == 128 ? kSw128 : (DI == 64 ? kSw64 : kSw32);
   static_assert(kTileBytes % 1024 == 0 && kQBytes % 1024 == 0, "tile alignment");
+  static_assert(kSmemAlloc <= 232448, "shared memory per CTA");
 };
 
 // Walks this CTA's slice of the flat (run, tile) list in order; every role runs its
@@ -235,12 +255,23 @@ struct ItemWalker {
   __device__ void advance() { ++i; }
 };
 
+// Page ids of 16 key tiles of run r from tile0 on (32 pages, one per lane; -2 past the
+// run's last page).
+__device__ __forceinline__ int load_page_window(const IdxArgs& a, const PlanView& pv, int r,
+                                                int tile0, int lane) {
+  const int nblk = (pv.maxpos[r] + kPage) / kPage;
+  const int lb = tile0 * 2 + lane;
+  return lb < nblk ? __ldg(&a.block_table[static_cast<size_t>(pv.seq[r]) * a.max_blocks + lb])
+                   : -2;
+}
+
 template <int DI, int HP, int RT>
 __global__ void __launch_bounds__(192, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap kmap, const IdxArgs a) {
   using C = IdxCfg<DI, HP, RT>;
   constexpr int NB = C::kNBuf;
   constexpr int S = C::kStages;
+  constexpr int NS = C::kScaleSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -251,9 +282,11 @@ __global__ void __launch_bounds__(192, 1)
   int* qtok = qpos + 2 * kRunTokens;
   int* qn = qtok + 2 * kRunTokens;  // tokens in the run held by each Q slot
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + S;
-  uint64_t* qfull = bars + 2 * S;
+  uint64_t* full = bars;            // [S] key tile landed
+  uint64_t* empty = full + S;       // [S] key tile consumed by the MMA
+  uint64_t* sfull = empty + S;      // [NS] scales landed, page ids written
+  uint64_t* sempty = sfull + NS;    // [NS] scales read by the epilogue
+  uint64_t* qfull = sempty + NS;
   uint64_t* qempty = qfull + 2;
   uint64_t* tfull = qempty + 2;   // [NB]
   uint64_t* tempty = tfull + NB;  // [NB]
@@ -264,17 +297,23 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   float* scales = reinterpret_cast<float*>(smem + C::kOffScale);
   int* pages = reinterpret_cast<int*>(smem + C::kOffPage);
+  int32_t* splan = reinterpret_cast<int32_t*>(smem + C::kOffPlan);
+  const bool inline_plan = a.plan == nullptr;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + 4);  // the MMA (keys) and the epilogue warps (scales)
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 4);
     }
     for (int q = 0; q < 2; ++q) {
-      mbar_init(&qfull[q], 1);
-      mbar_init(&qempty[q], 1 + 4);
+      mbar_init(&qfull[q], 4);      // the epilogue warps, which stage the query
+      mbar_init(&qempty[q], 1 + 4);  // the run's last MMA and the epilogue warps
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(&tfull[b], 1);
@@ -289,18 +328,57 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
+  } else if (warp == 1 && inline_plan) {
+    // One run per token, planned here from the token list.  The token list (like every
+    // other input) is complete before this grid starts: the prep kernel ahead of it lets
+    // it launch only after its own wait on everything earlier in the stream.
+    PlanView v = plan_view(splan, a.T);
+    int carry = 0;
+    for (int base = 0; base < a.T; base += 32) {
+      const int t = base + lane;
+      int ni = 0, seq = 0, pos = -1;
+      if (t < a.T) {
+        seq = a.tok_seq[t];
+        pos = a.tok_pos[t];
+        if (!(seq >= 0 && seq < a.batch && pos >= 0 && pos <= a.max_pos && pos < a.pos_cap)) {
+          if (blockIdx.x == 0) record_error(kErrBadIndex);
+          seq = 0;
+          pos = -1;  // no work for an invalid token
+        }
+        ni = (pos + kKeyTile) / kKeyTile;
+      }
+      int x = ni;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (t < a.T) {
+        v.tok0[t] = t;
+        v.ntok[t] = 1;
+        v.seq[t] = seq;
+        v.maxpos[t] = pos;
+        v.item0[t] = carry + x - ni;
+      }
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) {
+      v.item0[a.T] = carry;
+      v.hdr[0] = a.T;
+      v.hdr[1] = carry;
+    }
   }
   uint32_t* shist = reinterpret_cast<uint32_t*>(smem + C::kOffHist);
   if (a.hist)
-    for (int i = threadIdx.x; i < kRunTokens * 2048; i += blockDim.x) shist[i] = 0u;
+    for (int i = threadIdx.x; i < RT * 2048; i += blockDim.x) shist[i] = 0u;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  pdl_wait();  // the plan (and the zeroed histogram) come from the prep kernel
+  if (!inline_plan) pdl_wait();  // the plan comes from the prep kernel
   pdl_trigger();
-  PlanView pv = plan_view(a.plan, a.T);
+  PlanView pv = plan_view(inline_plan ? static_cast<void*>(splan) : a.plan, a.T);
   const int n_runs = pv.hdr[0];
   const int total = pv.hdr[1];
   const int i0 = static_cast<int>(static_cast<int64_t>(total) * blockIdx.x / gridDim.x);
@@ -317,81 +395,70 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    int n = 0;
-    int bt_run = -1, bt_lb0 = 0, my_pb = -2;
-    for (; wk.next(); wk.advance(), ++n) {
-      const int r = wk.r;
-      if (wk.new_run) {
-        const int slot = wk.rc & 1;
-        if (!mbar_wait_warp(&qempty[slot], ((wk.rc >> 1) & 1) ^ 1, abort_flag, 11)) break;
-        const int tok0 = pv.tok0[r], ntok = pv.ntok[r];
-        uint8_t* qb = qbuf + slot * C::kQBytes;
-        constexpr int kChunks = DI / 16;
-        for (int c = lane; c < ntok * HP * kChunks; c += 32) {
-          const int row = c / kChunks, cc = c % kChunks;
-          const int j = row / HP, h = row % HP;
-          uint4 val = make_uint4(0, 0, 0, 0);
-          if (h < a.n_idx_heads)
-            val = *reinterpret_cast<const uint4*>(
-                a.q8 + (static_cast<size_t>(tok0 + j) * a.n_idx_heads + h) * DI + cc * 16);
-          *reinterpret_cast<uint4*>(qb + swz_offset(row, cc * 16, DI)) = val;
+    // Eight key tiles per pass: lane 2j+h copies page h of tile j (its keys by TMA, its
+    // scales by a bulk copy), so one warp instruction issues sixteen copies.  Page ids come
+    // from the block table one pass ahead.
+    constexpr int B = C::kBatch;
+    const int n_items = i1 - i0;
+    const int j = lane >> 1, h = lane & 1;
+    int rl = lo;  // this lane's run cursor
+    auto page_for = [&](int nb) -> int {
+      const int i = i0 + nb + j;
+      if (lane >= 2 * B || i >= i1) return -2;
+      while (i >= pv.item0[rl + 1]) ++rl;
+      const int lb = (i - pv.item0[rl]) * 2 + h;
+      return lb < (pv.maxpos[rl] + kPage) / kPage
+                 ? __ldg(&a.block_table[static_cast<size_t>(pv.seq[rl]) * a.max_blocks + lb])
+                 : -2;  // -2: past the run's last block (not an error)
+    };
+    int next_pb = page_for(0);
+    int nb = 0;
+    for (; nb < n_items; nb += B) {
+      int pb = next_pb;
+      if (nb + B < n_items) next_pb = page_for(nb + B);
+      const int n = nb + j;
+      const bool act = lane < 2 * B && n < n_items;
+      const int stage = n % S, sc = n % NS;
+      bool ok = true;
+      if (act && h == 0)
+        ok = mbar_wait(&sempty[sc], ((n / NS) & 1) ^ 1, abort_flag, 21) &&
+             mbar_wait(&empty[stage], ((n / S) & 1) ^ 1, abort_flag, 12);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      if (act) {
+        if (pb != -2 && (pb < 0 || pb >= a.num_blocks)) {
+          record_error(kErrBadIndex);
+          pb = -1;
         }
-        for (int e = lane; e < ntok * HP; e += 32) {
-          const int j = e / HP, h = e % HP;
-          wq[(slot * kRunTokens + j) * HP + h] =
-              h < a.n_idx_heads
-                  ? a.w[static_cast<size_t>(tok0 + j) * a.n_idx_heads + h] * a.q_scale[tok0 + j]
-                  : 0.f;
-        }
-        if (lane < ntok) {
-          qpos[slot * kRunTokens + lane] = a.tok_pos[tok0 + lane];
-          qtok[slot * kRunTokens + lane] = tok0 + lane;
-        }
-        if (lane == 0) qn[slot] = ntok;
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&qfull[slot]);
+        if (pb == -2) pb = -1;
+        pages[sc * 2 + h] = pb;
       }
-      // block-table entries, 32 pages per warp-wide load
-      if (r != bt_run || wk.tile * 2 < bt_lb0 || wk.tile * 2 + 1 >= bt_lb0 + 32) {
-        bt_run = r;
-        bt_lb0 = wk.tile * 2;
-        const int nblk = (pv.maxpos[r] + kPage) / kPage;
-        const int lb = bt_lb0 + lane;
-        my_pb = lb < nblk ? a.block_table[static_cast<size_t>(pv.seq[r]) * a.max_blocks + lb]
-                          : -2;  // -2: past the run's last block (not an error)
-      }
-      const int pb0 = __shfl_sync(0xffffffffu, my_pb, wk.tile * 2 - bt_lb0);
-      const int pb1 = __shfl_sync(0xffffffffu, my_pb, wk.tile * 2 + 1 - bt_lb0);
-      const int stage = n % S;
-      if (!mbar_wait_warp(&empty[stage], ((n / S) & 1) ^ 1, abort_flag, 12)) break;
-      if (lane == 0 && !(a.inject && i0 == 0 && n == 0)) {
-        int pb[2] = {pb0, pb1};
-        uint32_t bytes = 0;
-        for (int h = 0; h < 2; ++h) {
-          if (pb[h] != -2 && (pb[h] < 0 || pb[h] >= a.num_blocks)) {
-            record_error(kErrBadIndex);
-            pb[h] = -1;
-          }
-          if (pb[h] == -2) pb[h] = -1;
-          pages[stage * 2 + h] = pb[h];
-          if (pb[h] >= 0) bytes += kPage * DI + kPage * 4;
+      const int valid = (pb >= 0) + (__shfl_xor_sync(0xffffffffu, pb, 1) >= 0);
+      const bool skip = a.inject && i0 == 0 && n == 0;  // test hook
+      __syncwarp();
+      if (act && h == 0 && !skip) {
+        if (valid) {
+          mbar_arrive_expect_tx(&sfull[sc], valid * kPage * 4);
+          mbar_arrive_expect_tx(&full[stage], valid * kPage * DI);
+        } else {
+          mbar_arrive(&sfull[sc]);
+          mbar_arrive(&full[stage]);
         }
-        if (bytes) mbar_arrive_expect_tx(&full[stage], bytes);
-        else mbar_arrive(&full[stage]);
-        for (int h = 0; h < 2; ++h)
-          if (pb[h] >= 0) {
-            tma_load_2d(ktiles + stage * C::kTileBytes + h * kPage * DI, &kmap, &full[stage], 0,
-                        pb[h] * kPage);
-            bulk_load(scales + stage * kKeyTile + h * kPage,
-                      a.k_scale + static_cast<size_t>(pb[h]) * kPage, kPage * 4, &full[stage]);
-          }
       }
       __syncwarp();
+      if (act && pb >= 0 && !skip) {
+        tma_load_2d(ktiles + stage * C::kTileBytes + h * kPage * DI, &kmap, &full[stage], 0,
+                    pb * kPage);
+        bulk_load(scales + sc * kKeyTile + h * kPage, a.k_scale + static_cast<size_t>(pb) * kPage,
+                  kPage * 4, &sfull[sc]);
+      }
     }
-    // let every issued TMA land before the CTA can exit
-    if (lane == 0)
-      for (int m = max(0, n - S); m < n; ++m) mbar_wait_drain(&full[m % S], (m / S) & 1);
+    // let every issued copy land before the CTA can exit
+    const int n_done = min(nb, n_items);
+    if (lane == 0) {
+      for (int m = max(0, n_done - S); m < n_done; ++m) mbar_wait_drain(&full[m % S], (m / S) & 1);
+      for (int m = max(0, n_done - NS); m < n_done; ++m)
+        mbar_wait_drain(&sfull[m % NS], (m / NS) & 1);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -428,9 +495,54 @@ __global__ void __launch_bounds__(192, 1)
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    const int etid = threadIdx.x - 64;  // 0..127
     int n = 0, n_flush = 0;
     int slot = 0, ntok = 0;
     float wreg[RT == 1 ? HP : 1];  // head weights of a one-token run, kept in registers
+    // The epilogue warps also stage each run's query (rows swizzled for the MMA, weights
+    // w * q_scale, positions): the first run's now, run rc+1's on entering run rc.
+    auto fill_q = [&](int r, int qs) {
+      constexpr int kChunks = DI / 16;
+      const int tok0 = pv.tok0[r], nt = pv.ntok[r];
+      uint8_t* qb = qbuf + qs * C::kQBytes;
+      const int pieces = nt * HP * kChunks;
+      for (int c0 = 0; c0 < pieces; c0 += 8 * 128) {
+        uint4 val[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int c = c0 + u * 128 + etid;
+          const int rw = c / kChunks, cc = c % kChunks;
+          const int jj = rw / HP, hh = rw % HP;
+          val[u] = make_uint4(0, 0, 0, 0);
+          if (c < pieces && hh < a.n_idx_heads)
+            val[u] = __ldg(reinterpret_cast<const uint4*>(
+                a.q8 + (static_cast<size_t>(tok0 + jj) * a.n_idx_heads + hh) * DI + cc * 16));
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int c = c0 + u * 128 + etid;
+          if (c < pieces)
+            *reinterpret_cast<uint4*>(qb + swz_offset(c / kChunks, (c % kChunks) * 16, DI)) =
+                val[u];
+        }
+      }
+      for (int e = etid; e < nt * HP; e += 128) {
+        const int jj = e / HP, hh = e % HP;
+        wq[(qs * kRunTokens + jj) * HP + hh] =
+            hh < a.n_idx_heads
+                ? a.w[static_cast<size_t>(tok0 + jj) * a.n_idx_heads + hh] * a.q_scale[tok0 + jj]
+                : 0.f;
+      }
+      if (etid < nt) {
+        qpos[qs * kRunTokens + etid] = a.tok_pos[tok0 + etid];
+        qtok[qs * kRunTokens + etid] = tok0 + etid;
+      }
+      if (etid == 0) qn[qs] = nt;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qfull[qs]);
+    };
+    if (i0 < i1) fill_q(lo, 0);
     for (; wk.next(); wk.advance(), ++n) {
       if (wk.new_run) {
         slot = wk.rc & 1;
@@ -440,16 +552,24 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int h = 0; h < HP; ++h) wreg[h] = wq[slot * kRunTokens * HP + h];
         }
+        // the next run with work in this slice goes to the other slot once run rc-1 is
+        // done with it (its last MMA and this epilogue)
+        int rn = wk.r + 1;
+        const int inext = pv.item0[wk.r + 1];
+        if (inext < i1) {
+          while (pv.item0[rn + 1] <= inext) ++rn;
+          if (!mbar_wait_warp(&qempty[slot ^ 1], (((wk.rc + 1) >> 1) & 1) ^ 1, abort_flag, 11))
+            break;
+          fill_q(rn, slot ^ 1);
+        }
       }
-      const int ab = n % NB;
+      const int ab = n % NB, sc = n % NS;
       if (!mbar_wait_warp(&tfull[ab], (n / NB) & 1, abort_flag, 17)) break;
       tc_fence_after();
       const int s = wk.tile * kKeyTile + row;
-      const int stage = n % S;
-      // the stage's scales and page ids (complete: the MMA already waited for it)
-      if (!mbar_wait_warp(&full[stage], (n / S) & 1, abort_flag, 18)) break;
-      const float ks = pages[stage * 2 + (row >> 6)] >= 0 ? scales[stage * kKeyTile + row]
-                                                           : __int_as_float(0x7fc00000);
+      if (!mbar_wait_warp(&sfull[sc], (n / NS) & 1, abort_flag, 18)) break;
+      const float ks = pages[sc * 2 + (row >> 6)] >= 0 ? scales[sc * kKeyTile + row]
+                                                        : __int_as_float(0x7fc00000);
       for (int j = 0; j < (RT == 1 ? 1 : ntok); ++j) {
         float x[HP];
         const uint32_t taddr =
@@ -486,13 +606,15 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&tempty[ab]);
-        mbar_arrive(&empty[stage]);
+        mbar_arrive(&sempty[sc]);
         if (wk.last_of_run) mbar_arrive(&qempty[slot]);
       }
       if (a.hist && wk.last_of_run) {
-        // this CTA is done with the run: add its histogram to the global one.  The four
-        // epilogue warps meet on hist_full, each flushes (and clears) a quarter of the
-        // bins, and they meet again on hist_free before any bin is reused.
+        // this CTA is done with the run: add its histogram to the global one (zeroed by
+        // the prep kernel, hence the wait for it).  The four epilogue warps meet on
+        // hist_full, each flushes (and clears) a quarter of the bins, and they meet again
+        // on hist_free before any bin is reused.
+        pdl_wait();
         __syncwarp();
         if (lane == 0) mbar_arrive(hist_full);
         if (!mbar_wait_warp(hist_full, n_flush & 1, abort_flag, 19)) break;
@@ -514,6 +636,8 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
 
+  // this grid completes only after the prep kernel (so after everything before it)
+  if (inline_plan) pdl_wait();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -554,14 +678,18 @@ static cudaError_t launch_indexer_t(const IndexerLaunch& L, const CUtensorMap& m
   a.block_table = L.cache->block_table;
   a.max_blocks = L.cache->max_blocks_per_seq;
   a.num_blocks = L.cache->num_blocks;
+  a.tok_seq = L.queries->tok_seq;
   a.tok_pos = L.queries->tok_pos;
+  a.batch = L.cache->batch;
+  a.max_pos = L.queries->max_pos;
+  a.pos_cap = L.cache->max_blocks_per_seq * kPage;
   a.q8 = L.q8;
   a.q_scale = L.q_scale;
   a.w = L.w;
   a.n_idx_heads = L.n_idx_heads;
   a.logits = L.logits;
   a.ld = L.ld_logits;
-  a.plan = L.ws;
+  a.plan = RT == 1 && L.queries->n_tokens <= kInlinePlanMax ? nullptr : L.ws;
   a.T = L.queries->n_tokens;
   a.hist = L.hist;
   a.inject = take_injection(1);
@@ -577,9 +705,12 @@ cudaError_t launch_indexer(const IndexerLaunch& L) {
   // one query token per sequence on average (decode): runs of one token, which lets the
   // kernel keep eight accumulator buffers in TMEM; otherwise runs of up to four tokens
   const int RT = T <= c->batch ? 1 : kRunTokens;
+  // with runs of one token and few tokens the indexer plans for itself; the prep kernel
+  // then only zeroes (and orders this launch after everything earlier in the stream)
+  const bool inline_plan = RT == 1 && T <= kInlinePlanMax;
   cudaError_t e = launch_pdl(indexer_prep_kernel, dim3(1), dim3(1024), 0, L.stream, q->tok_seq,
                              q->tok_pos, T, c->batch, q->max_pos, c->max_blocks_per_seq * kPage,
-                             L.ws, L.zero, L.zero_words, RT);
+                             inline_plan ? nullptr : L.ws, L.zero, L.zero_words, RT);
   if (e != cudaSuccess) return e;
 
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
