@@ -96,6 +96,21 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
+// try_wait that may suspend the thread for up to kWaitSleepNs while the phase is open (it
+// resumes as soon as the phase completes), so waiting warps leave the issue slots of their
+// scheduler to the warps that have work.
+constexpr uint32_t kWaitSleepNs = 20000;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitSleepNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of parity `parity`.  On timeout: records kErrTimeout and the
 // wait site, sets *abort (shared) and returns false.  Also returns false at once if
 // *abort is set.
@@ -104,7 +119,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(bar, parity)) return true;
   const long long c0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     if (*abort) return false;
     if (clock64() - c0 > kWaitBudgetCycles) {
       record_timeout(site);
@@ -139,9 +154,18 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
 // Bounded wait that ignores the abort flag (draining in-flight copies before exit).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const long long c0 = clock64();
-  while (!mbar_try_wait(bar, parity))
+  while (!mbar_try_wait_sleep(bar, parity))
     if (clock64() - c0 > kWaitBudgetCycles) return false;
   return true;
+}
+
+// ------------------------------------------------------------------ named barriers
+// Hardware barrier `id` (1..15; 0 is __syncthreads) over `count` threads, a multiple of 32.
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_barrier_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ------------------------------------------------------------------ proxies / fences

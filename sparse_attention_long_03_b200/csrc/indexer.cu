@@ -13,11 +13,13 @@
 // without any cross-thread traffic.  Keys stream from the paged cache with TMA (one
 // 64-token page per box, swizzled for the MMA), through a multi-stage mbarrier ring.
 //
-//   warp 0      producer: key pages by TMA and their scales by bulk copy, up to eight key
-//               tiles per pass (one page per lane)
-//   warp 1      one thread issues tcgen05.mma (kind::f8f6f4) and tcgen05.commit
-//   warps 2..5  epilogue: tcgen05.ld -> ReLU . w -> logits (coalesced fp32 stores); they
-//               also stage each run's query rows (manual swizzled stores) one run ahead
+//   warp 0      producer: key pages by TMA and their scales by bulk copy, up to four key
+//               tiles per pass (one per lane); it also plans decode batches itself
+//   warps 1,10  one thread each issues tcgen05.mma (kind::f8f6f4) and tcgen05.commit,
+//               for alternate key tiles
+//   warps 2..9  epilogue, two warps per TMEM lane quarter on alternate key tiles:
+//               tcgen05.ld -> ReLU . w -> logits (coalesced fp32 stores); they also stage
+//               each run's query rows (manual swizzled stores) one run ahead
 //
 // A small planner kernel first groups the query tokens into runs of up to 4 tokens of
 // the same sequence (they share every key tile) and lays the (run, key tile) work items
@@ -192,8 +194,16 @@ struct IdxArgs {
 
 // Query tokens up to which one-token runs are planned inside the indexer kernel.
 constexpr int kInlinePlanMax = 64;
-// Key tiles the producer warp issues per pass (two pages each, one per lane), at most.
-constexpr int kProducerBatch = 8;
+// Warps: producer, two MMA issuers, eight epilogue warps (two per TMEM lane quarter).
+constexpr int kEpiWarps = 8;
+// warp 10 is a second MMA issuer (odd key tiles)
+constexpr int kMmaWarp2 = 2 + kEpiWarps;
+constexpr int kIdxThreads = (3 + kEpiWarps) * 32;
+// Registers are split over the SM's four schedulers and warps are dealt to them in turn,
+// so with eleven warps three schedulers hold three: bound registers as for twelve warps.
+constexpr int kIdxThreadsBound = 12 * 32;
+// Key tiles the producer warp issues per pass (one per lane), at most.
+constexpr int kProducerBatch = 4;
 
 __host__ __device__ constexpr int pow2ceil(int x) {
   int p = 32;
@@ -236,20 +246,37 @@ struct IdxCfg {
 };
 
 // Walks this CTA's slice of the flat (run, tile) list in order; every role runs its
-// own copy so they agree on run boundaries without talking to each other.
+// own copy so they agree on run boundaries without talking to each other.  The current
+// run's item range is held in registers: a step reads the plan only when it leaves a run.
 struct ItemWalker {
   const int32_t* item0;
   int i, i1, r, rc;
+  int run_start, run_end;  // item0[r], item0[r + 1]
   bool new_run, last_of_run;
   int tile;
+  __device__ void init(const int32_t* it0, int first, int end, int run) {
+    item0 = it0;
+    i = first;
+    i1 = end;
+    r = run;
+    rc = -1;
+    run_start = first < end ? item0[run] : 0;
+    run_end = first < end ? item0[run + 1] : 0;
+  }
   __device__ bool next() {
     if (i >= i1) return false;
-    const int prev = r;
-    while (i >= item0[r + 1]) ++r;
-    new_run = (rc < 0) || (r != prev);
+    new_run = rc < 0;
+    if (i >= run_end) {  // into the next run with items (empty runs are skipped)
+      do {
+        ++r;
+        run_start = run_end;
+        run_end = item0[r + 1];
+      } while (i >= run_end);
+      new_run = true;
+    }
     if (new_run) ++rc;
-    tile = i - item0[r];
-    last_of_run = (i + 1 >= i1) || (i + 1 >= item0[r + 1]);
+    tile = i - run_start;
+    last_of_run = (i + 1 >= i1) || (i + 1 >= run_end);
     return true;
   }
   __device__ void advance() { ++i; }
@@ -266,7 +293,7 @@ __device__ __forceinline__ int load_page_window(const IdxArgs& a, const PlanView
 }
 
 template <int DI, int HP, int RT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kIdxThreadsBound, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap kmap, const IdxArgs a) {
   using C = IdxCfg<DI, HP, RT>;
   constexpr int NB = C::kNBuf;
@@ -312,130 +339,146 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&sempty[s], 4);
     }
     for (int q = 0; q < 2; ++q) {
-      mbar_init(&qfull[q], 4);      // the epilogue warps, which stage the query
-      mbar_init(&qempty[q], 1 + 4);  // the run's last MMA and the epilogue warps
+      mbar_init(&qfull[q], kEpiWarps);      // the epilogue warps, which stage the query
+      mbar_init(&qempty[q], 2 + kEpiWarps);  // both MMA issuers and the epilogue warps
     }
     for (int b = 0; b < NB; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4);
     }
-    mbar_init(drain, 1);
-    mbar_init(hist_full, 4);
-    mbar_init(hist_free, 4);
+    mbar_init(drain, 2);
+    mbar_init(hist_full, kEpiWarps);
+    mbar_init(hist_free, kEpiWarps);
     *abort_flag = 0;
     fence_barrier_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
-  } else if (warp == 1 && inline_plan) {
-    // One run per token, planned here from the token list.  The token list (like every
-    // other input) is complete before this grid starts: the prep kernel ahead of it lets
-    // it launch only after its own wait on everything earlier in the stream.
-    PlanView v = plan_view(splan, a.T);
-    int carry = 0;
-    for (int base = 0; base < a.T; base += 32) {
-      const int t = base + lane;
-      int ni = 0, seq = 0, pos = -1;
-      if (t < a.T) {
-        seq = a.tok_seq[t];
-        pos = a.tok_pos[t];
-        if (!(seq >= 0 && seq < a.batch && pos >= 0 && pos <= a.max_pos && pos < a.pos_cap)) {
-          if (blockIdx.x == 0) record_error(kErrBadIndex);
-          seq = 0;
-          pos = -1;  // no work for an invalid token
-        }
-        ni = (pos + kKeyTile) / kKeyTile;
-      }
-      int x = ni;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (t < a.T) {
-        v.tok0[t] = t;
-        v.ntok[t] = 1;
-        v.seq[t] = seq;
-        v.maxpos[t] = pos;
-        v.item0[t] = carry + x - ni;
-      }
-      carry += __shfl_sync(0xffffffffu, x, 31);
-    }
-    if (lane == 0) {
-      v.item0[a.T] = carry;
-      v.hdr[0] = a.T;
-      v.hdr[1] = carry;
-    }
   }
   uint32_t* shist = reinterpret_cast<uint32_t*>(smem + C::kOffHist);
   if (a.hist)
     for (int i = threadIdx.x; i < RT * 2048; i += blockDim.x) shist[i] = 0u;
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
 
-  if (!inline_plan) pdl_wait();  // the plan comes from the prep kernel
-  pdl_trigger();
-  PlanView pv = plan_view(inline_plan ? static_cast<void*>(splan) : a.plan, a.T);
-  const int n_runs = pv.hdr[0];
-  const int total = pv.hdr[1];
-  const int i0 = static_cast<int>(static_cast<int64_t>(total) * blockIdx.x / gridDim.x);
-  const int i1 = static_cast<int>(static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x);
+  // This CTA's slice of the flat (run, tile) list: items [i0, i1), the first in run lo.
+  PlanView pv{};
+  int i0 = 0, i1 = 0, lo = 0;
+  auto find_slice = [&]() {
+    pv = plan_view(inline_plan ? static_cast<void*>(splan) : a.plan, a.T);
+    const int n_runs = pv.hdr[0];
+    const int total = pv.hdr[1];
+    i0 = static_cast<int>(static_cast<int64_t>(total) * blockIdx.x / gridDim.x);
+    i1 = static_cast<int>(static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x);
+    lo = 0;
+    int hi = n_runs;  // item0[lo] <= i0 < item0[hi]
+    while (i0 < i1 && hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pv.item0[mid] <= i0) lo = mid;
+      else hi = mid;
+    }
+  };
 
-  // run containing item i0
-  int lo = 0, hi = n_runs;  // item0[lo] <= i0 < item0[hi]
-  while (i0 < i1 && hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (pv.item0[mid] <= i0) lo = mid;
-    else hi = mid;
-  }
-  ItemWalker wk{pv.item0, i0, i1, lo, -1, false, false, 0};
+  // The epilogue warps stage each run's query (rows swizzled for the MMA, weights
+  // w * q_scale, positions): the first run's before the CTA barrier, run rc+1's on entering
+  // run rc.  Every load is issued before any store.
+  const int etid = threadIdx.x - 64;  // 0..255 in the epilogue warps
+  auto fill_q = [&](int r, int qs) {
+    constexpr int kChunks = DI / 16;
+    constexpr int kE = kEpiWarps * 32;
+    const int tok0 = pv.tok0[r], nt = pv.ntok[r];
+    uint8_t* qb = qbuf + qs * C::kQBytes;
+    const int pieces = nt * HP * kChunks;
+    float wv = 0.f;
+    int tp = 0;
+    for (int c0 = 0; c0 < pieces; c0 += 4 * kE) {
+      uint4 val[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * kE + etid;
+        const int rw = c / kChunks, cc = c % kChunks;
+        const int jj = rw / HP, hh = rw % HP;
+        val[u] = make_uint4(0, 0, 0, 0);
+        if (c < pieces && hh < a.n_idx_heads)
+          val[u] = __ldg(reinterpret_cast<const uint4*>(
+              a.q8 + (static_cast<size_t>(tok0 + jj) * a.n_idx_heads + hh) * DI + cc * 16));
+      }
+      if (c0 == 0) {
+        const int jj = etid / HP, hh = etid % HP;
+        if (etid < nt * HP && hh < a.n_idx_heads)
+          wv = a.w[static_cast<size_t>(tok0 + jj) * a.n_idx_heads + hh] * a.q_scale[tok0 + jj];
+        if (etid < nt) tp = a.tok_pos[tok0 + etid];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u * kE + etid;
+        if (c < pieces)
+          *reinterpret_cast<uint4*>(qb + swz_offset(c / kChunks, (c % kChunks) * 16, DI)) = val[u];
+      }
+    }
+    if (etid < nt * HP) wq[qs * kRunTokens * HP + etid] = wv;  // [token][head]
+    if (etid < nt) {
+      qpos[qs * kRunTokens + etid] = tp;
+      qtok[qs * kRunTokens + etid] = tok0 + etid;
+    }
+    if (etid == 0) qn[qs] = nt;
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&qfull[qs]);
+  };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // Eight key tiles per pass: lane 2j+h copies page h of tile j (its keys by TMA, its
-    // scales by a bulk copy), so one warp instruction issues sixteen copies.  Page ids come
-    // from the block table one pass ahead.
-    constexpr int B = C::kBatch;
-    const int n_items = i1 - i0;
-    const int j = lane >> 1, h = lane & 1;
-    int rl = lo;  // this lane's run cursor
-    auto page_for = [&](int nb) -> int {
-      const int i = i0 + nb + j;
-      if (lane >= 2 * B || i >= i1) return -2;
-      while (i >= pv.item0[rl + 1]) ++rl;
-      const int lb = (i - pv.item0[rl]) * 2 + h;
-      return lb < (pv.maxpos[rl] + kPage) / kPage
-                 ? __ldg(&a.block_table[static_cast<size_t>(pv.seq[rl]) * a.max_blocks + lb])
-                 : -2;  // -2: past the run's last block (not an error)
-    };
-    int next_pb = page_for(0);
-    int nb = 0;
-    for (; nb < n_items; nb += B) {
-      int pb = next_pb;
-      if (nb + B < n_items) next_pb = page_for(nb + B);
-      const int n = nb + j;
-      const bool act = lane < 2 * B && n < n_items;
+  // ---------------------------------------------------------------- producer (warp 0)
+  // B key tiles per pass, one per lane: each lane copies its tile's two scale rows (bulk)
+  // and its two key pages (TMA), the scale copies of a pass queued ahead of its key pages.
+  // Page ids come from the block table one pass ahead.  The producer plans (decode), finds
+  // its slice and issues the first passes before the CTA barrier below.
+  constexpr int B = C::kBatch;
+  int n_items = 0, rl = 0, nb = 0, cur0 = -2, cur1 = -2;
+  // this lane's run cursor: run rl covers items [rl_start, rl_end), nblk pages of the
+  // block-table row bt
+  int rl_start = 0, rl_end = 0, rl_nblk = 0;
+  const int32_t* rl_bt = nullptr;
+  auto enter_run = [&]() {
+    rl_start = pv.item0[rl];
+    rl_end = pv.item0[rl + 1];
+    rl_nblk = (pv.maxpos[rl] + kPage) / kPage;
+    rl_bt = a.block_table + static_cast<size_t>(pv.seq[rl]) * a.max_blocks;
+  };
+  auto pages_of = [&](int base, int& q0, int& q1) {
+    q0 = q1 = -2;  // -2: past the run's last block (not an error)
+    const int n = base + lane;
+    if (lane >= B || n >= n_items) return;
+    const int i = i0 + n;
+    if (i >= rl_end) {
+      do ++rl;
+      while (i >= pv.item0[rl + 1]);
+      enter_run();
+    }
+    const int lb = (i - rl_start) * 2;
+    if (lb < rl_nblk) q0 = __ldg(rl_bt + lb);
+    if (lb + 1 < rl_nblk) q1 = __ldg(rl_bt + lb + 1);
+  };
+  auto produce = [&](int limit) -> bool {
+    for (; nb < limit; nb += B) {
+      const int n = nb + lane;
+      const bool act = lane < B && n < n_items;
+      int pb[2] = {cur0, cur1};
+      pages_of(nb + B, cur0, cur1);
       const int stage = n % S, sc = n % NS;
       bool ok = true;
-      if (act && h == 0)
+      if (act)
         ok = mbar_wait(&sempty[sc], ((n / NS) & 1) ^ 1, abort_flag, 21) &&
              mbar_wait(&empty[stage], ((n / S) & 1) ^ 1, abort_flag, 12);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      const bool go = act && !(a.inject && i0 == 0 && n == 0);  // test hook
+      int valid = 0;
       if (act) {
-        if (pb != -2 && (pb < 0 || pb >= a.num_blocks)) {
-          record_error(kErrBadIndex);
-          pb = -1;
+        for (int h = 0; h < 2; ++h) {
+          if (pb[h] != -2 && (pb[h] < 0 || pb[h] >= a.num_blocks)) {
+            record_error(kErrBadIndex);
+            pb[h] = -1;
+          }
+          if (pb[h] == -2) pb[h] = -1;
+          pages[sc * 2 + h] = pb[h];
+          valid += pb[h] >= 0;
         }
-        if (pb == -2) pb = -1;
-        pages[sc * 2 + h] = pb;
       }
-      const int valid = (pb >= 0) + (__shfl_xor_sync(0xffffffffu, pb, 1) >= 0);
-      const bool skip = a.inject && i0 == 0 && n == 0;  // test hook
-      __syncwarp();
-      if (act && h == 0 && !skip) {
+      if (go) {
         if (valid) {
           mbar_arrive_expect_tx(&sfull[sc], valid * kPage * 4);
           mbar_arrive_expect_tx(&full[stage], valid * kPage * DI);
@@ -443,15 +486,96 @@ __global__ void __launch_bounds__(192, 1)
           mbar_arrive(&sfull[sc]);
           mbar_arrive(&full[stage]);
         }
-      }
-      __syncwarp();
-      if (act && pb >= 0 && !skip) {
-        tma_load_2d(ktiles + stage * C::kTileBytes + h * kPage * DI, &kmap, &full[stage], 0,
-                    pb * kPage);
-        bulk_load(scales + sc * kKeyTile + h * kPage, a.k_scale + static_cast<size_t>(pb) * kPage,
-                  kPage * 4, &sfull[sc]);
+        for (int h = 0; h < 2; ++h)
+          if (pb[h] >= 0)
+            bulk_load(scales + sc * kKeyTile + h * kPage,
+                      a.k_scale + static_cast<size_t>(pb[h]) * kPage, kPage * 4, &sfull[sc]);
+        for (int h = 0; h < 2; ++h)
+          if (pb[h] >= 0)
+            tma_load_2d(ktiles + stage * C::kTileBytes + h * kPage * DI, &kmap, &full[stage], 0,
+                        pb[h] * kPage);
       }
     }
+    return true;
+  };
+  bool producing = true;
+  if (warp == 0) {
+    __syncwarp();  // the barriers lane 0 initialised
+    if (inline_plan) {
+      // One run per token, planned here from the token list.  The token list (like every
+      // other input) is complete before this grid starts: the prep kernel ahead of it
+      // lets it launch only after its own wait on everything earlier in the stream.
+      PlanView v = plan_view(splan, a.T);
+      int carry = 0;
+      for (int base = 0; base < a.T; base += 32) {
+        const int t = base + lane;
+        int ni = 0, seq = 0, pos = -1;
+        if (t < a.T) {
+          seq = a.tok_seq[t];
+          pos = a.tok_pos[t];
+          if (!(seq >= 0 && seq < a.batch && pos >= 0 && pos <= a.max_pos && pos < a.pos_cap)) {
+            if (blockIdx.x == 0) record_error(kErrBadIndex);
+            seq = 0;
+            pos = -1;  // no work for an invalid token
+          }
+          ni = (pos + kKeyTile) / kKeyTile;
+        }
+        int x = ni;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (t < a.T) {
+          v.tok0[t] = t;
+          v.ntok[t] = 1;
+          v.seq[t] = seq;
+          v.maxpos[t] = pos;
+          v.item0[t] = carry + x - ni;
+        }
+        carry += __shfl_sync(0xffffffffu, x, 31);
+      }
+      if (lane == 0) {
+        v.item0[a.T] = carry;
+        v.hdr[0] = a.T;
+        v.hdr[1] = carry;
+      }
+      __syncwarp();
+    } else {
+      pdl_wait();  // the plan comes from the prep kernel
+    }
+    named_barrier_arrive(1, 32 + kEpiWarps * 32);  // the plan is readable
+    find_slice();
+    n_items = i1 - i0;
+    rl = lo;
+    if (n_items > 0) enter_run();
+    pages_of(0, cur0, cur1);
+    // stages and scale slots are all free: no wait can block before the barrier
+    constexpr int kPre = ((S < NS ? S : NS) / B) * B;
+    producing = produce(n_items < kPre ? n_items : kPre);
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  } else if (warp < kMmaWarp2) {
+    named_barrier_sync(1, 32 + kEpiWarps * 32);  // warp 0 has published the plan
+    if (!inline_plan) pdl_wait();                // the plan comes from the prep kernel
+    find_slice();
+    if (i0 < i1) fill_q(lo, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp == 1 || warp == kMmaWarp2) {
+    if (!inline_plan) pdl_wait();  // the plan comes from the prep kernel
+    find_slice();
+  }
+  pdl_trigger();
+  ItemWalker wk;
+  wk.init(pv.item0, i0, i1, lo);
+
+  if (warp == 0) {
+    if (producing) produce(n_items);
     // let every issued copy land before the CTA can exit
     const int n_done = min(nb, n_items);
     if (lane == 0) {
@@ -459,32 +583,38 @@ __global__ void __launch_bounds__(192, 1)
       for (int m = max(0, n_done - NS); m < n_done; ++m)
         mbar_wait_drain(&sfull[m % NS], (m / NS) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == kMmaWarp2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two threads (in warps on different schedulers) issue alternate key tiles; each
+    // commits its own tiles and, at every run's end, the run's query slot.
     if (lane == 0) {
+      const int mpar = warp == 1 ? 0 : 1;
       int n = 0;
       int slot = 0;
+      uint32_t N = 0;
       for (; wk.next(); wk.advance(), ++n) {
         const int r = wk.r;
         if (wk.new_run) {
           slot = wk.rc & 1;
+          N = static_cast<uint32_t>(pv.ntok[r] * HP);
           if (!mbar_wait(&qfull[slot], (wk.rc >> 1) & 1, abort_flag, 13)) break;
         }
-        const int ab = n % NB;
-        if (!mbar_wait(&tempty[ab], ((n / NB) & 1) ^ 1, abort_flag, 14)) break;
-        const int stage = n % S;
-        if (!mbar_wait(&full[stage], (n / S) & 1, abort_flag, 15)) break;
-        tc_fence_after();
-        const uint32_t N = static_cast<uint32_t>(pv.ntok[r] * HP);
-        const uint32_t idesc = instr_desc(128, N, 0, 0, 0, 0);
-        const uint32_t a_base = smem_u32(ktiles + stage * C::kTileBytes);
-        const uint32_t b_base = smem_u32(qbuf + slot * C::kQBytes);
+        if ((n & 1) == mpar) {
+          const int ab = n % NB;
+          if (!mbar_wait(&tempty[ab], ((n / NB) & 1) ^ 1, abort_flag, 14)) break;
+          const int stage = n % S;
+          if (!mbar_wait(&full[stage], (n / S) & 1, abort_flag, 15)) break;
+          tc_fence_after();
+          const uint32_t idesc = instr_desc(128, N, 0, 0, 0, 0);
+          const uint32_t a_base = smem_u32(ktiles + stage * C::kTileBytes);
+          const uint32_t b_base = smem_u32(qbuf + slot * C::kQBytes);
 #pragma unroll
-        for (int ks = 0; ks < DI / 32; ++ks)
-          mma_f8(tmem + ab * C::kNC, smem_desc(a_base + ks * 32, 16, 8 * DI, C::kSwz),
-                 smem_desc(b_base + ks * 32, 16, 8 * DI, C::kSwz), idesc, ks > 0 ? 1u : 0u);
-        mma_commit(&empty[stage]);
-        mma_commit(&tfull[ab]);
+          for (int ks = 0; ks < DI / 32; ++ks)
+            mma_f8(tmem + ab * C::kNC, smem_desc(a_base + ks * 32, 16, 8 * DI, C::kSwz),
+                   smem_desc(b_base + ks * 32, 16, 8 * DI, C::kSwz), idesc, ks > 0 ? 1u : 0u);
+          mma_commit(&empty[stage]);
+          mma_commit(&tfull[ab]);
+        }
         if (wk.last_of_run) mma_commit(&qempty[slot]);
       }
       mma_commit(drain);
@@ -492,70 +622,24 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------------------ epilogue (warps 2..9)
+    // Two warps per TMEM lane quarter take alternate key tiles.  Each walks every item (to
+    // track runs) and releases a run's query slot, and meets the others for the histogram
+    // flush, when it passes the run's last item.
     const int quarter = warp & 3;
+    const int par = (warp - 2) >> 2;  // items n with n % 2 == par
     const int row = quarter * 32 + lane;
-    const int etid = threadIdx.x - 64;  // 0..127
     int n = 0, n_flush = 0;
     int slot = 0, ntok = 0;
-    float wreg[RT == 1 ? HP : 1];  // head weights of a one-token run, kept in registers
-    // The epilogue warps also stage each run's query (rows swizzled for the MMA, weights
-    // w * q_scale, positions): the first run's now, run rc+1's on entering run rc.
-    auto fill_q = [&](int r, int qs) {
-      constexpr int kChunks = DI / 16;
-      const int tok0 = pv.tok0[r], nt = pv.ntok[r];
-      uint8_t* qb = qbuf + qs * C::kQBytes;
-      const int pieces = nt * HP * kChunks;
-      for (int c0 = 0; c0 < pieces; c0 += 8 * 128) {
-        uint4 val[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int c = c0 + u * 128 + etid;
-          const int rw = c / kChunks, cc = c % kChunks;
-          const int jj = rw / HP, hh = rw % HP;
-          val[u] = make_uint4(0, 0, 0, 0);
-          if (c < pieces && hh < a.n_idx_heads)
-            val[u] = __ldg(reinterpret_cast<const uint4*>(
-                a.q8 + (static_cast<size_t>(tok0 + jj) * a.n_idx_heads + hh) * DI + cc * 16));
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int c = c0 + u * 128 + etid;
-          if (c < pieces)
-            *reinterpret_cast<uint4*>(qb + swz_offset(c / kChunks, (c % kChunks) * 16, DI)) =
-                val[u];
-        }
-      }
-      for (int e = etid; e < nt * HP; e += 128) {
-        const int jj = e / HP, hh = e % HP;
-        wq[(qs * kRunTokens + jj) * HP + hh] =
-            hh < a.n_idx_heads
-                ? a.w[static_cast<size_t>(tok0 + jj) * a.n_idx_heads + hh] * a.q_scale[tok0 + jj]
-                : 0.f;
-      }
-      if (etid < nt) {
-        qpos[qs * kRunTokens + etid] = a.tok_pos[tok0 + etid];
-        qtok[qs * kRunTokens + etid] = tok0 + etid;
-      }
-      if (etid == 0) qn[qs] = nt;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&qfull[qs]);
-    };
-    if (i0 < i1) fill_q(lo, 0);
     for (; wk.next(); wk.advance(), ++n) {
       if (wk.new_run) {
         slot = wk.rc & 1;
         if (!mbar_wait_warp(&qfull[slot], (wk.rc >> 1) & 1, abort_flag, 16)) break;
         ntok = qn[slot];
-        if constexpr (RT == 1) {
-#pragma unroll
-          for (int h = 0; h < HP; ++h) wreg[h] = wq[slot * kRunTokens * HP + h];
-        }
         // the next run with work in this slice goes to the other slot once run rc-1 is
-        // done with it (its last MMA and this epilogue)
+        // done with it (its last MMA and every epilogue warp)
         int rn = wk.r + 1;
-        const int inext = pv.item0[wk.r + 1];
+        const int inext = wk.run_end;
         if (inext < i1) {
           while (pv.item0[rn + 1] <= inext) ++rn;
           if (!mbar_wait_warp(&qempty[slot ^ 1], (((wk.rc + 1) >> 1) & 1) ^ 1, abort_flag, 11))
@@ -563,75 +647,75 @@ __global__ void __launch_bounds__(192, 1)
           fill_q(rn, slot ^ 1);
         }
       }
-      const int ab = n % NB, sc = n % NS;
-      if (!mbar_wait_warp(&tfull[ab], (n / NB) & 1, abort_flag, 17)) break;
-      tc_fence_after();
-      const int s = wk.tile * kKeyTile + row;
-      if (!mbar_wait_warp(&sfull[sc], (n / NS) & 1, abort_flag, 18)) break;
-      const float ks = pages[sc * 2 + (row >> 6)] >= 0 ? scales[sc * kKeyTile + row]
-                                                        : __int_as_float(0x7fc00000);
-      for (int j = 0; j < (RT == 1 ? 1 : ntok); ++j) {
-        float x[HP];
-        const uint32_t taddr =
-            tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::kNC + j * HP;
-        if constexpr (HP % 32 == 0) {
-#pragma unroll
-          for (int c = 0; c < HP / 32; ++c) tmem_ld32(taddr + c * 32, x + c * 32);
-        } else {
-          tmem_ld16(taddr, x);
-        }
-        tmem_wait_ld();
-        if (s <= qpos[slot * kRunTokens + j]) {
-          float acc0 = 0.f, acc1 = 0.f;
-          if constexpr (RT == 1) {
-#pragma unroll
-            for (int h = 0; h < HP; h += 2) {
-              acc0 = fmaf(fmaxf(x[h], 0.f), wreg[h], acc0);
-              acc1 = fmaf(fmaxf(x[h + 1], 0.f), wreg[h + 1], acc1);
-            }
-          } else {
-            const float* wv = wq + (slot * kRunTokens + j) * HP;
-#pragma unroll
-            for (int h = 0; h < HP; h += 2) {
-              acc0 = fmaf(fmaxf(x[h], 0.f), wv[h], acc0);
-              acc1 = fmaf(fmaxf(x[h + 1], 0.f), wv[h + 1], acc1);
-            }
-          }
-          const float v = (acc0 + acc1) * ks;
-          a.logits[static_cast<int64_t>(qtok[slot * kRunTokens + j]) * a.ld + s] = v;
-          if (a.hist) atomicAdd(&shist[j * 2048 + (float_to_ordered(v) >> 21)], 1u);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&tempty[ab]);
-        mbar_arrive(&sempty[sc]);
-        if (wk.last_of_run) mbar_arrive(&qempty[slot]);
-      }
-      if (a.hist && wk.last_of_run) {
-        // this CTA is done with the run: add its histogram to the global one (zeroed by
-        // the prep kernel, hence the wait for it).  The four epilogue warps meet on
-        // hist_full, each flushes (and clears) a quarter of the bins, and they meet again
-        // on hist_free before any bin is reused.
-        pdl_wait();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(hist_full);
-        if (!mbar_wait_warp(hist_full, n_flush & 1, abort_flag, 19)) break;
+      if ((n & 1) == par) {
+        const int ab = n % NB, sc = n % NS;
+        if (!mbar_wait_warp(&tfull[ab], (n / NB) & 1, abort_flag, 17)) break;
+        tc_fence_after();
+        const int s = wk.tile * kKeyTile + row;
+        if (!mbar_wait_warp(&sfull[sc], (n / NS) & 1, abort_flag, 18)) break;
+        const float ks = pages[sc * 2 + (row >> 6)] >= 0 ? scales[sc * kKeyTile + row]
+                                                          : __int_as_float(0x7fc00000);
         for (int j = 0; j < ntok; ++j) {
-          uint32_t* gh = a.hist + static_cast<size_t>(qtok[slot * kRunTokens + j]) * 2048;
-          for (int d = quarter * 512 + lane; d < (quarter + 1) * 512; d += 32) {
-            const uint32_t c = shist[j * 2048 + d];
-            if (c) {
-              atomicAdd(&gh[d], c);
-              shist[j * 2048 + d] = 0u;
+          float x[HP];
+          const uint32_t taddr =
+              tmem + (static_cast<uint32_t>(quarter * 32) << 16) + ab * C::kNC + j * HP;
+          if constexpr (HP % 32 == 0) {
+#pragma unroll
+            for (int c = 0; c < HP / 32; ++c) tmem_ld32(taddr + c * 32, x + c * 32);
+          } else {
+            tmem_ld16(taddr, x);
+          }
+          tmem_wait_ld();
+          if (s <= qpos[slot * kRunTokens + j]) {
+            const float4* wv = reinterpret_cast<const float4*>(wq + (slot * kRunTokens + j) * HP);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int h = 0; h < HP; h += 4) {
+              const float4 w4 = wv[h / 4];
+              acc[0] = fmaf(fmaxf(x[h], 0.f), w4.x, acc[0]);
+              acc[1] = fmaf(fmaxf(x[h + 1], 0.f), w4.y, acc[1]);
+              acc[2] = fmaf(fmaxf(x[h + 2], 0.f), w4.z, acc[2]);
+              acc[3] = fmaf(fmaxf(x[h + 3], 0.f), w4.w, acc[3]);
             }
+            const float v = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * ks;
+            a.logits[static_cast<int64_t>(qtok[slot * kRunTokens + j]) * a.ld + s] = v;
+            if (a.hist) atomicAdd(&shist[j * 2048 + (float_to_ordered(v) >> 21)], 1u);
           }
         }
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(hist_free);
-        if (!mbar_wait_warp(hist_free, n_flush & 1, abort_flag, 20)) break;
-        ++n_flush;
+        if (lane == 0) {
+          mbar_arrive(&tempty[ab]);
+          mbar_arrive(&sempty[sc]);
+        }
+      }
+      if (wk.last_of_run) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qempty[slot]);
+        if (a.hist) {
+          // this CTA is done with the run: add its histogram to the global one (zeroed by
+          // the prep kernel, hence the wait for it).  The eight epilogue warps meet on
+          // hist_full, each flushes (and clears) an eighth of the bins, and they meet
+          // again on hist_free before any bin is reused.
+          pdl_wait();
+          if (lane == 0) mbar_arrive(hist_full);
+          if (!mbar_wait_warp(hist_full, n_flush & 1, abort_flag, 19)) break;
+          const int ew = warp - 2;
+          for (int j = 0; j < ntok; ++j) {
+            uint32_t* gh = a.hist + static_cast<size_t>(qtok[slot * kRunTokens + j]) * 2048;
+            for (int d = ew * 256 + lane; d < (ew + 1) * 256; d += 32) {
+              const uint32_t c = shist[j * 2048 + d];
+              if (c) {
+                atomicAdd(&gh[d], c);
+                shist[j * 2048 + d] = 0u;
+              }
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(hist_free);
+          if (!mbar_wait_warp(hist_free, n_flush & 1, abort_flag, 20)) break;
+          ++n_flush;
+        }
       }
     }
   }
@@ -640,7 +724,7 @@ __global__ void __launch_bounds__(192, 1)
   if (inline_plan) pdl_wait();
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {  // the allocating warp
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -693,7 +777,7 @@ static cudaError_t launch_indexer_t(const IndexerLaunch& L, const CUtensorMap& m
   a.T = L.queries->n_tokens;
   a.hist = L.hist;
   a.inject = take_injection(1);
-  return launch_pdl(indexer_kernel<DI, HP, RT>, dim3(grid), dim3(192), C::kSmemAlloc, L.stream,
+  return launch_pdl(indexer_kernel<DI, HP, RT>, dim3(grid), dim3(kIdxThreads), C::kSmemAlloc, L.stream,
                     map, a);
 }
 
