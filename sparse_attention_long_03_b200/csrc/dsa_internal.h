@@ -70,7 +70,7 @@ struct TopkDecodeLayout {
   int64_t zero_words;  // hist + arrive, from the start of the region
   int32_t* counts;
   int32_t* scr_a;
-  int32_t* scr_b;
+  int2* scr_b;
 };
 size_t topk_decode_ws_bytes(int32_t T, int64_t ld, int chunks);
 int topk_decode_chunks(int32_t T, int32_t max_pos);

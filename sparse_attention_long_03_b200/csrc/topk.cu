@@ -12,7 +12,8 @@
 // a higher bucket is already selected and is written out at once; the elements of the
 // threshold bucket are gathered (in position order) into a shared candidate list, and
 // the two remaining digits run on that list only.  All writes are ordered compactions
-// (warp ballots + a block scan), so the result is deterministic.
+// (each thread classifies a run of consecutive elements, one block scan per round), so
+// the result is deterministic.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -189,29 +190,61 @@ __device__ void select_bucket(TopkSmem* sm, int nb, int k_rem) {
   __syncthreads();
 }
 
-// One ordered pass: class A elements go to outA[baseA + rank]; class B elements with
-// rank < limitB go to the B sink.  cls(key) -> 0 none, 1 A, 2 B.
-template <class Src, class Cls, class SinkB>
-__device__ int2 ordered_pass(TopkSmem* sm, const Src& src, int n, Cls cls, int32_t* outA,
-                             int baseA, SinkB sinkB, int limitB) {
+// Block-wide exclusive scan of two per-thread counters.
+__device__ __forceinline__ void thread_scan_two(TopkSmem* sm, int a, int b, int* off_a,
+                                                int* off_b, int* tot_a, int* tot_b) {
   const int lane = threadIdx.x & 31;
-  int run_a = 0, run_b = 0;
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    int c = 0;
-    uint32_t key = 0;
-    if (i < n) {
-      key = src.key(i);
-      c = cls(key);
+  int ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ya = __shfl_up_sync(0xffffffffu, ia, o), yb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia += ya;
+      ib += yb;
     }
-    const uint32_t ba = __ballot_sync(0xffffffffu, c == 1);
-    const uint32_t bb = __ballot_sync(0xffffffffu, c == 2);
+  }
+  int wa, wb, ta, tb;
+  scan_two(sm, __shfl_sync(0xffffffffu, ia, 31), __shfl_sync(0xffffffffu, ib, 31), &wa, &wb, &ta,
+           &tb);
+  *off_a = wa + ia - a;
+  *off_b = wb + ib - b;
+  *tot_a = ta;
+  *tot_b = tb;
+}
+
+// The same ordered compaction with one block scan per round of blockDim.x * E elements:
+// thread t owns E consecutive elements (E odd, so a warp's shared-memory reads of its
+// elements fall in 32 different banks), counts its two classes, and after the scan writes
+// its elements in position order.
+template <int E, class Src, class Cls, class SinkA, class SinkB>
+__device__ int2 ordered_pass_seg(TopkSmem* sm, const Src& src, int n, Cls cls, SinkA sinkA,
+                                 SinkB sinkB, int limitB) {
+  static_assert(E % 2 == 1 && E <= 31, "odd element count per thread");
+  int run_a = 0, run_b = 0;
+  for (int base = 0; base < n; base += static_cast<int>(blockDim.x) * E) {
+    const int i0 = base + static_cast<int>(threadIdx.x) * E;
+    uint32_t keys[E];
+    uint32_t ma = 0, mb = 0;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      keys[j] = 0;
+      if (i0 + j < n) {
+        keys[j] = src.key(i0 + j);
+        const int c = cls(keys[j]);
+        if (c == 1) ma |= 1u << j;
+        if (c == 2) mb |= 1u << j;
+      }
+    }
     int off_a, off_b, tot_a, tot_b;
-    scan_two(sm, __popc(ba), __popc(bb), &off_a, &off_b, &tot_a, &tot_b);
-    if (c == 1) outA[baseA + run_a + off_a + __popc(ba & lanemask_lt())] = src.index(i);
-    if (c == 2) {
-      const int rb = run_b + off_b + __popc(bb & lanemask_lt());
-      if (rb < limitB) sinkB(rb, key, src.index(i));
+    thread_scan_two(sm, __popc(ma), __popc(mb), &off_a, &off_b, &tot_a, &tot_b);
+    int ra = run_a + off_a, rb = run_b + off_b;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      if ((ma >> j) & 1u) sinkA(ra++, keys[j], src.index(i0 + j));
+      if ((mb >> j) & 1u) {
+        if (rb < limitB) sinkB(rb, keys[j], src.index(i0 + j));
+        ++rb;
+      }
     }
     run_a += tot_a;
     run_b += tot_b;
@@ -233,9 +266,10 @@ __device__ void finish_candidates(TopkSmem* sm, const Src& cs, int n_cand, uint3
   const uint32_t thr = (b1 << 21) | (b2 << 10) | static_cast<uint32_t>(sm->sel[0]);
   const int need_eq = k2 - above2 - sm->sel[1];
   int32_t* eq_out = out + (k2 - need_eq);
-  ordered_pass(
-      sm, cs, n_cand, [thr](uint32_t key) { return key > thr ? 1 : (key == thr ? 2 : 0); }, out,
-      0, [eq_out](int r, uint32_t, int idx) { eq_out[r] = idx; }, need_eq);
+  ordered_pass_seg<3>(
+      sm, cs, n_cand, [thr](uint32_t key) { return key > thr ? 1 : (key == thr ? 2 : 0); },
+      [out](int r, uint32_t, int idx) { out[r] = idx; },
+      [eq_out](int r, uint32_t, int idx) { eq_out[r] = idx; }, need_eq);
 }
 
 template <class Src>
@@ -249,10 +283,10 @@ __device__ void select_from(TopkSmem* sm, const Src& src, int n, int k, int32_t*
   const int k2 = k - above1;
   if (n_cand <= kTopkCand) {
     // higher buckets are final; gather the threshold bucket in position order
-    ordered_pass(
+    ordered_pass_seg<7>(
         sm, src, n,
-        [b1](uint32_t key) { return (key >> 21) > b1 ? 1 : ((key >> 21) == b1 ? 2 : 0); }, out,
-        0,
+        [b1](uint32_t key) { return (key >> 21) > b1 ? 1 : ((key >> 21) == b1 ? 2 : 0); },
+        [out](int r, uint32_t, int idx) { out[r] = idx; },
         [sm](int r, uint32_t key, int idx) {
           sm->cand_key[r] = key;
           sm->cand_idx[r] = idx;
@@ -270,8 +304,9 @@ __device__ void select_from(TopkSmem* sm, const Src& src, int n, int k, int32_t*
     const uint32_t thr = (b1 << 21) | (b2 << 10) | static_cast<uint32_t>(sm->sel[0]);
     const int need_eq = k2 - above2 - sm->sel[1];
     int32_t* eq_out = out + (k - need_eq);
-    ordered_pass(
-        sm, src, n, [thr](uint32_t key) { return key > thr ? 1 : (key == thr ? 2 : 0); }, out, 0,
+    ordered_pass_seg<7>(
+        sm, src, n, [thr](uint32_t key) { return key > thr ? 1 : (key == thr ? 2 : 0); },
+        [out](int r, uint32_t, int idx) { out[r] = idx; },
         [eq_out](int r, uint32_t, int idx) { eq_out[r] = idx; }, need_eq);
   }
 }
@@ -340,8 +375,24 @@ struct TopkDecodeWs {
   uint32_t* arrive;      // [T] arrival counters, zero on entry
   int32_t* counts;       // [T][chunks][2]
   int32_t* scr_a;        // [T][ld] finals, at each chunk's position range
-  int32_t* scr_b;        // [T][ld] candidates, same
+  int2* scr_b;           // [T][ld] candidates (position, ordered key), same
 };
+
+// Threshold-bucket candidates read back by the finishing CTA: (position, key) pairs.
+struct CandPairs {
+  const int2* list;
+  __device__ uint32_t key(int i) const { return static_cast<uint32_t>(list[i].y); }
+  __device__ int index(int i) const { return list[i].x; }
+};
+
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+
+// Chunk elements each thread classifies per round of the decode pass (odd, see
+// ordered_pass_seg).
+constexpr int kDecPerThread = 7;
 
 __global__ void __launch_bounds__(kTopkDecThreads, 1)
     topk_decode_kernel(const float* __restrict__ logits, int64_t ld,
@@ -368,6 +419,13 @@ __global__ void __launch_bounds__(kTopkDecThreads, 1)
     return;
   }
   const float* row = logits + static_cast<int64_t>(t) * ld;
+  const int c0 = static_cast<int>(static_cast<int64_t>(n) * c / chunks);
+  const int c1 = static_cast<int>(static_cast<int64_t>(n) * (c + 1) / chunks);
+  // this CTA's chunk: asynchronous copies into shared memory, in flight while the
+  // histogram is read and the threshold bucket chosen
+  float* ck = reinterpret_cast<float*>(topk_smem_raw + kTopkSmemBase);
+  for (int i = threadIdx.x; i < c1 - c0; i += blockDim.x) cp_async_4(ck + i, row + c0 + i);
+  cp_async_commit();
   for (int b = threadIdx.x; b < 2048; b += blockDim.x)
     sm->hist[b] = ws.hist[static_cast<size_t>(t) * 2048 + b];
   __syncthreads();
@@ -375,18 +433,22 @@ __global__ void __launch_bounds__(kTopkDecThreads, 1)
   const uint32_t b1 = static_cast<uint32_t>(sm->sel[0]);
   const int above1 = sm->sel[1];
   const int n_cand = sm->sel[2];
-  const int c0 = static_cast<int>(static_cast<int64_t>(n) * c / chunks);
-  const int c1 = static_cast<int>(static_cast<int64_t>(n) * (c + 1) / chunks);
-  int32_t* sa = ws.scr_a + static_cast<int64_t>(t) * ld;
-  int32_t* sb = ws.scr_b + static_cast<int64_t>(t) * ld;
-  // this CTA's chunk, read once into shared memory with every load in flight
-  uint32_t* ck = reinterpret_cast<uint32_t*>(topk_smem_raw + kTopkSmemBase);
-  for (int i = threadIdx.x; i < c1 - c0; i += blockDim.x) ck[i] = float_to_ordered(row[c0 + i]);
+  cp_async_wait<0>();
   __syncthreads();
-  const int2 cnt = ordered_pass(
-      sm, RowCachedOff{ck, c0}, c1 - c0,
-      [b1](uint32_t key) { return (key >> 21) > b1 ? 1 : ((key >> 21) == b1 ? 2 : 0); }, sa, c0,
-      [sb, c0](int r, uint32_t, int i) { sb[c0 + r] = i; }, c1 - c0);
+  int32_t* sa = ws.scr_a + static_cast<int64_t>(t) * ld;
+  int2* sb = ws.scr_b + static_cast<int64_t>(t) * ld;
+  struct ChunkKeys {
+    const float* v;
+    int off;
+    __device__ uint32_t key(int i) const { return float_to_ordered(v[i]); }
+    __device__ int index(int i) const { return off + i; }
+  };
+  const int2 cnt = ordered_pass_seg<kDecPerThread>(
+      sm, ChunkKeys{ck, c0}, c1 - c0,
+      [b1](uint32_t key) { return (key >> 21) > b1 ? 1 : ((key >> 21) == b1 ? 2 : 0); },
+      [sa, c0](int r, uint32_t, int i) { sa[c0 + r] = i; },
+      [sb, c0](int r, uint32_t key, int i) { sb[c0 + r] = make_int2(i, static_cast<int>(key)); },
+      c1 - c0);
   if (threadIdx.x == 0) {
     ws.counts[(static_cast<size_t>(t) * chunks + c) * 2] = cnt.x;
     ws.counts[(static_cast<size_t>(t) * chunks + c) * 2 + 1] = cnt.y;
@@ -397,19 +459,34 @@ __global__ void __launch_bounds__(kTopkDecThreads, 1)
   __syncthreads();
   if (!sm->sel[3]) return;
   __threadfence();
-  // ---- the last CTA of this row finishes it.  Every step below issues its global loads
-  // in parallel (no loop over chunks with a round trip per chunk).
-  for (int cc = threadIdx.x; cc < chunks; cc += blockDim.x) {
-    sm->pre_a[cc + 1] = ws.counts[(static_cast<size_t>(t) * chunks + cc) * 2];
-    sm->pre_b[cc + 1] = ws.counts[(static_cast<size_t>(t) * chunks + cc) * 2 + 1];
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    sm->pre_a[0] = 0;
-    sm->pre_b[0] = 0;
-    for (int cc = 0; cc < chunks; ++cc) {
-      sm->pre_a[cc + 1] += sm->pre_a[cc];
-      sm->pre_b[cc + 1] += sm->pre_b[cc];
+  // ---- the last CTA of this row finishes it; every step issues its global loads together.
+  if (threadIdx.x < 32) {
+    // prefix sums of the per-chunk counts (chunks <= kTopkMaxChunks = 4 x 32)
+    const int lane = threadIdx.x;
+    int carry_a = 0, carry_b = 0;
+    for (int base = 0; base < chunks; base += 32) {
+      const int cc = base + lane;
+      const int va = cc < chunks ? ws.counts[(static_cast<size_t>(t) * chunks + cc) * 2] : 0;
+      const int vb = cc < chunks ? ws.counts[(static_cast<size_t>(t) * chunks + cc) * 2 + 1] : 0;
+      int ia = va, ib = vb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ya = __shfl_up_sync(0xffffffffu, ia, o), yb = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) {
+          ia += ya;
+          ib += yb;
+        }
+      }
+      if (cc < chunks) {
+        sm->pre_a[cc + 1] = carry_a + ia;
+        sm->pre_b[cc + 1] = carry_b + ib;
+      }
+      carry_a += __shfl_sync(0xffffffffu, ia, 31);
+      carry_b += __shfl_sync(0xffffffffu, ib, 31);
+    }
+    if (lane == 0) {
+      sm->pre_a[0] = 0;
+      sm->pre_b[0] = 0;
     }
   }
   __syncthreads();
@@ -424,45 +501,82 @@ __global__ void __launch_bounds__(kTopkDecThreads, 1)
     return lo;
   };
   auto chunk_start = [&](int cc) { return static_cast<int>(static_cast<int64_t>(n) * cc / chunks); };
-  for (int g = threadIdx.x; g < sm->pre_a[chunks]; g += blockDim.x) {
-    const int cc = chunk_of(sm->pre_a, g);
-    out[g] = sa[chunk_start(cc) + g - sm->pre_a[cc]];
-  }
-  // the counts actually gathered decide (they equal the histogram's when all is well)
   const int got_a = sm->pre_a[chunks], got_b = sm->pre_b[chunks];
   const int k2 = k - got_a;
+  // the counts actually gathered decide (they equal the histogram's when all is well)
   if (got_a != above1 || got_b != n_cand || k2 < 1 || k2 > got_b) {
     if (threadIdx.x == 0) record_error(kErrBadIndex);
-    for (int i = got_a + threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
+    for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
     return;
   }
+  // the finals, in chunk order: all loads first, then the stores
+  constexpr int kFin = (kMaxTopK + kTopkDecThreads - 1) / kTopkDecThreads;
+  {
+    int32_t v[kFin];
+#pragma unroll
+    for (int u = 0; u < kFin; ++u) {
+      const int g = u * kTopkDecThreads + threadIdx.x;
+      v[u] = 0;
+      if (g < got_a) {
+        const int cc = chunk_of(sm->pre_a, g);
+        v[u] = sa[chunk_start(cc) + g - sm->pre_a[cc]];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kFin; ++u) {
+      const int g = u * kTopkDecThreads + threadIdx.x;
+      if (g < got_a) out[g] = v[u];
+    }
+  }
   if (got_b <= kTopkCand) {
-    for (int g = threadIdx.x; g < got_b; g += blockDim.x) {
-      const int cc = chunk_of(sm->pre_b, g);
-      const int p = sb[chunk_start(cc) + g - sm->pre_b[cc]];
-      sm->cand_idx[g] = p;
-      sm->cand_key[g] = float_to_ordered(row[p]);
+    for (int g0 = 0; g0 < got_b; g0 += 4 * kTopkDecThreads) {
+      int2 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int g = g0 + u * kTopkDecThreads + threadIdx.x;
+        v[u] = make_int2(0, 0);
+        if (g < got_b) {
+          const int cc = chunk_of(sm->pre_b, g);
+          v[u] = sb[chunk_start(cc) + g - sm->pre_b[cc]];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int g = g0 + u * kTopkDecThreads + threadIdx.x;
+        if (g < got_b) {
+          sm->cand_idx[g] = v[u].x;
+          sm->cand_key[g] = static_cast<uint32_t>(v[u].y);
+        }
+      }
     }
     __syncthreads();
     finish_candidates(sm, RowCand{sm->cand_key, sm->cand_idx}, got_b, b1, k2, out + got_a);
   } else {
-    // too many candidates for shared memory: compact them into the (now free) finals
-    // scratch and resolve from global memory
-    __syncthreads();
-    for (int g = threadIdx.x; g < got_b; g += blockDim.x) {
-      const int cc = chunk_of(sm->pre_b, g);
-      sa[g] = sb[chunk_start(cc) + g - sm->pre_b[cc]];
+    // too many candidates for shared memory: compact them (position, key) into the front
+    // of this row's candidate scratch (in place: entry g moves to g or lower) and resolve
+    // from global memory
+    for (int g0 = 0; g0 < got_b; g0 += blockDim.x) {  // same trip count in every thread
+      const int g = g0 + threadIdx.x;
+      int2 e = make_int2(0, 0);
+      if (g < got_b) {
+        const int cc = chunk_of(sm->pre_b, g);
+        e = sb[chunk_start(cc) + g - sm->pre_b[cc]];
+      }
+      __syncthreads();
+      if (g < got_b) sb[g] = e;
+      __syncthreads();
     }
     __threadfence_block();
     __syncthreads();
-    finish_candidates(sm, CandGlobal{row, sa}, got_b, b1, k2, out + got_a);
+    finish_candidates(sm, CandPairs{sb}, got_b, b1, k2, out + got_a);
   }
 }
 
 size_t topk_decode_ws_bytes(int32_t T, int64_t ld, int chunks) {
   auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   return al(static_cast<size_t>(T) * 2048 * 4) + al(static_cast<size_t>(T) * 4) +
-         al(static_cast<size_t>(T) * chunks * 8) + 2 * al(static_cast<size_t>(T) * ld * 4);
+         al(static_cast<size_t>(T) * chunks * 8) + al(static_cast<size_t>(T) * ld * 4) +
+         al(static_cast<size_t>(T) * ld * 8);
 }
 
 // Largest chunk a CTA of the decode kernel reads (rows are at most max_pos + 1 long).
@@ -494,7 +608,7 @@ TopkDecodeLayout topk_decode_layout(void* ws, int32_t T, int64_t ld, int chunks)
   p += al(static_cast<size_t>(T) * chunks * 8);
   L.scr_a = reinterpret_cast<int32_t*>(p);
   p += al(static_cast<size_t>(T) * ld * 4);
-  L.scr_b = reinterpret_cast<int32_t*>(p);
+  L.scr_b = reinterpret_cast<int2*>(p);
   return L;
 }
 
