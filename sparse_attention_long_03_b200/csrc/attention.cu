@@ -177,17 +177,24 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         rows[u] = resolve_row(v, pos, seq, a, warp == 5);
       }
       uint8_t* tb = tiles + b * kTile;
-      const int pieces = kBN * 8 * nc;  // (row, chunk, 16-byte piece)
-      for (int p = pl; p < pieces; p += kProducers * 32) {
-        const int c = p / (kBN * 8), rem = p % (kBN * 8), r = rem >> 3, c16 = rem & 7;
+      // lane pl copies the 16-byte piece c16 = pl % 8 of every chunk of tile rows
+      // pl / 8, pl / 8 + 8, ...: one row lookup per row, then one copy per chunk
+      const int c16 = pl & 7;
+#pragma unroll 1
+      for (int r = pl >> 3; r < kBN; r += kProducers * 4) {
         // the physical row of tile row r sits in lane r % 32 (slot r < 32: rows[0], else rows[1])
         const int r0 = __shfl_sync(0xffffffffu, rows[0], r & 31);
         const int r1 = __shfl_sync(0xffffffffu, rows[1], r & 31);
         const int row = (r >> 5) ? r1 : r0;
-        const int d0 = c * 64 + c16 * 8;
-        const int valid = row >= 0 ? max(0, min(8, a.d_kv - d0)) : 0;
-        const uint16_t* src = valid ? a.kv + static_cast<size_t>(row) * a.d_kv + d0 : a.kv;
-        cp_async_16(tb + c * kKVChunk + swz_offset(r, c16 * 16, 128), src, valid * 2);
+        uint8_t* dst = tb + swz_offset(r, c16 * 16, 128);
+        const uint16_t* src = a.kv + static_cast<size_t>(row < 0 ? 0 : row) * a.d_kv + c16 * 8;
+#pragma unroll
+        for (int c = 0; c < kMaxChunks; ++c) {
+          if (c < nc) {
+            const int valid = row >= 0 ? max(0, min(8, a.d_kv - (c * 64 + c16 * 8))) : 0;
+            cp_async_16(dst + c * kKVChunk, valid ? src + c * 64 : a.kv, valid * 2);
+          }
+        }
       }
       cp_async_commit();
       cp_async_wait<0>();
@@ -220,7 +227,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
       const uint32_t idesc_s = instr_desc(128, kBN, 1, 1, 0, 0);
-      const uint32_t idesc_pv = instr_desc(128, 64, 1, 1, 0, 1);
+      const uint32_t idesc_pv = instr_desc(128, 64 * a.nvg, 1, 1, 0, 1);
       const uint32_t tile_base = smem_u32(tiles), q_base = smem_u32(qring), p_base = smem_u32(ps);
       bool ok = true;
       int qn = 0;
@@ -230,16 +237,16 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         fence_proxy_async_smem();
         const uint32_t tb = tile_base + (j & 1) * kTile;
         // P = P_hi + P_lo (both bf16): the second product restores the bits a single
-        // bf16 P would lose, so the value weights are exact to ~2^-17
-        for (int vc = 0; vc < a.nvg; ++vc)
+        // bf16 P would lose, so the value weights are exact to ~2^-17.  One MMA covers all
+        // of this CTA's value chunks: N = nvg * 64, the B operand's 64-wide MN atoms (the
+        // value chunks) kKVChunk apart.
 #pragma unroll
-          for (int ks = 0; ks < kBN / 16; ++ks)
+        for (int ks = 0; ks < kBN / 16; ++ks)
 #pragma unroll
-            for (int part = 0; part < 2; ++part)
-              mma_bf16(tmem_o + vc * 64,
-                       smem_desc(p_base + part * kPBytes + ks * 32, 16, 1024, kSw128),
-                       smem_desc(tb + (vc0 + vc) * kKVChunk + ks * 2048, kKVChunk, 1024, kSw128),
-                       idesc_pv, (j > 0 || ks > 0 || part > 0) ? 1u : 0u);
+          for (int part = 0; part < 2; ++part)
+            mma_bf16(tmem_o, smem_desc(p_base + part * kPBytes + ks * 32, 16, 1024, kSw128),
+                     smem_desc(tb + vc0 * kKVChunk + ks * 2048, kKVChunk, 1024, kSw128),
+                     idesc_pv, (j > 0 || ks > 0 || part > 0) ? 1u : 0u);
         mma_commit(&tile_empty[j & 1]);
         mma_commit(pv_done);
         return true;
