@@ -20,12 +20,15 @@
 // MMA).  P enters as two bf16 parts hi + lo (the A operand from shared memory), so the
 // probabilities keep ~16 significant bits.  Rescaling of O is lazy: the running max used
 // for P only moves when it grows by more than 2^8.  Long selections are split over several
-// CTAs (split-KV) and merged by LSE in a second kernel.
+// CTAs (split-KV) and merged by LSE in a second kernel; the partial outputs, each
+// normalised by its own softmax sum and so bounded by the largest |value| entry, travel as
+// fp16 (2^-12 relative rounding, well below the bf16 output's own).
 //
 //   warps 0..3  softmax: online softmax, P, O rescale, output (one head row per thread)
 //   warp 4      one thread issues tcgen05.mma for S and for P.V, and the commits
 //   warps 5..6  gatherers: each 64-key tile's selected rows, all 9 chunks, by cp.async
 //   warp 7      one thread streams the query's 64-dim chunks by TMA through a 3-slot ring
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include "dsa_common.cuh"
@@ -46,7 +49,7 @@ constexpr int kOffQ = kOffTile + 2 * kTile;
 constexpr int kOffP = kOffQ + kQRing * kQChunk;  // P_hi, then P_lo (bf16, 128 x 64 each)
 constexpr int kPBytes = 128 * 128;
 constexpr int kOffBar = kOffP + 2 * kPBytes;
-constexpr int kNumBars = 24;
+constexpr int kNumBars = 32;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmem = kOffMisc + 16;
 constexpr int kSmemAlloc = kSmem + 1024;
@@ -57,6 +60,8 @@ constexpr int kProducers = 2;                    // gathering warps 5..6
 constexpr int kThreads = (6 + kProducers) * 32;  // + the query-chunk warp 7: 8 warps, since
                                                  // registers are granted per 4 warps
 static_assert(kTile % 1024 == 0 && kQChunk % 1024 == 0, "swizzle atoms");
+// the split epilogue stages 128 rows of up to kMaxVC * 64 fp16 (+16 bytes) in the tiles
+static_assert(128 * (kMaxVC * 128 + 16) <= 2 * kTile, "staged partial rows");
 static_assert(kSmemAlloc <= 232448, "shared memory");
 }  // namespace attn
 
@@ -79,7 +84,7 @@ struct AttnArgs {
   int32_t nvg;        // value chunks per group
   uint16_t* out;
   float* lse;
-  float* part_o;    // [T, splits, H, d_v] fp32 (splits > 1)
+  uint16_t* part_o;  // [T, splits, H, d_v] fp16 (splits > 1), each normalised by its own sum
   float* part_lse;  // [T, splits, H]
   int inject;       // test hook: CTA (0, 0) skips its first query-chunk arrival
 };
@@ -107,9 +112,9 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* tile_full = bars;           // [2] gathered tile landed (96 producer lanes)
-  uint64_t* tile_empty = bars + 2;      // [2] P.V of that tile done (MMA commit)
-  uint64_t* q_full = bars + 4;          // [kQRing] query chunk landed (TMA)
+  uint64_t* chunk_full = bars;                // [kMaxChunks] chunk c of the pair's tiles landed
+  uint64_t* tile_empty = bars + kMaxChunks;  // [2] P.V of that tile done (MMA commit)
+  uint64_t* q_full = tile_empty + 2;         // [kQRing] query chunk landed (TMA)
   uint64_t* q_empty = q_full + kQRing;  // [kQRing] score MMA done with it (MMA commit)
   uint64_t* s_full = q_empty + kQRing;  // [2]
   uint64_t* s_free = s_full + 2;        // [2]
@@ -136,7 +141,6 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&tile_full[i], kProducers * 32);
       mbar_init(&tile_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
@@ -145,6 +149,7 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
+    for (int c = 0; c < kMaxChunks; ++c) mbar_init(&chunk_full[c], kProducers * 32);
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
     mbar_init(drain, 1);
@@ -166,40 +171,62 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
     // Each tile: 64 selected rows x nc chunks x 8 pieces of 16 B, all issued with cp.async
     // in one go by the 64 lanes, then one wait for the whole tile.
     const int pl = threadIdx.x - 5 * 32;  // 0..63
-    bool ok = true;
-    for (int i = 0; ok && i < n_tiles; ++i) {
-      const int b = i & 1;
-      if (!mbar_wait_warp(&tile_empty[b], ((i >> 1) & 1) ^ 1, abort_flag, 42)) break;
+    const int c16 = pl & 7;
+    // Lane pl copies 16-byte piece c16 = pl % 8 of tile rows r_j = pl / 8 + 8 j (j < 8).
+    // Their swizzled slots differ only by j * 1024: r_j & 7 is the same for every j.
+    const int rbase = pl >> 3;
+    const uint32_t lane_dst = rbase * 128 + ((c16 ^ (rbase & 7)) << 4);
+    constexpr int kRowsPerLane = kBN / (kProducers * 4);
+    static_assert(kRowsPerLane == 8, "gather lane mapping");
+    // physical rows of this lane's tile rows (-1: empty or invalid slot)
+    auto lane_rows = [&](int i, int* prow) {
       int rows[2];
       for (int u = 0; u < 2; ++u) {
         const int slot = k0 + i * kBN + lane + 32 * u;
         const int v = slot < k1 ? a.idx[static_cast<size_t>(t) * a.k + slot] : -1;
         rows[u] = resolve_row(v, pos, seq, a, warp == 5);
       }
-      uint8_t* tb = tiles + b * kTile;
-      // lane pl copies the 16-byte piece c16 = pl % 8 of every chunk of tile rows
-      // pl / 8, pl / 8 + 8, ...: one row lookup per row, then one copy per chunk
-      const int c16 = pl & 7;
-#pragma unroll 1
-      for (int r = pl >> 3; r < kBN; r += kProducers * 4) {
+#pragma unroll
+      for (int j = 0; j < kRowsPerLane; ++j) {
+        const int r = rbase + 8 * j;
         // the physical row of tile row r sits in lane r % 32 (slot r < 32: rows[0], else rows[1])
         const int r0 = __shfl_sync(0xffffffffu, rows[0], r & 31);
         const int r1 = __shfl_sync(0xffffffffu, rows[1], r & 31);
-        const int row = (r >> 5) ? r1 : r0;
-        uint8_t* dst = tb + swz_offset(r, c16 * 16, 128);
-        const uint16_t* src = a.kv + static_cast<size_t>(row < 0 ? 0 : row) * a.d_kv + c16 * 8;
+        prow[j] = (r >> 5) ? r1 : r0;
+      }
+    };
+    // Tiles go in pairs (the scores of a pair share one pass over the query).  A pair is
+    // gathered chunk-major, one cp.async group per 64-dim chunk of both tiles, and each
+    // chunk is announced on its own barrier as soon as it has landed, so the score MMAs
+    // of chunk 0 can start while the later chunks are still in flight.
+    for (int g = 0; 2 * g < n_tiles; ++g) {
+      const int ia = 2 * g;
+      const bool has_b = ia + 1 < n_tiles;
+      if (!mbar_wait_warp(&tile_empty[0], (g & 1) ^ 1, abort_flag, 42)) break;
+      if (has_b && !mbar_wait_warp(&tile_empty[1], (g & 1) ^ 1, abort_flag, 42)) break;
+      int prow[2][kRowsPerLane];
+      lane_rows(ia, prow[0]);
+      if (has_b) lane_rows(ia + 1, prow[1]);
+      for (int c = 0; c < nc; ++c) {
+        const int valid = max(0, min(8, a.d_kv - (c * 64 + c16 * 8)));
+        for (int tb = 0; tb < (has_b ? 2 : 1); ++tb) {
+          uint8_t* dst = tiles + tb * kTile + c * kKVChunk + lane_dst;
 #pragma unroll
-        for (int c = 0; c < kMaxChunks; ++c) {
-          if (c < nc) {
-            const int valid = row >= 0 ? max(0, min(8, a.d_kv - (c * 64 + c16 * 8))) : 0;
-            cp_async_16(dst + c * kKVChunk, valid ? src + c * 64 : a.kv, valid * 2);
+          for (int j = 0; j < kRowsPerLane; ++j) {
+            const int row = prow[tb][j];
+            const int vb = row >= 0 ? valid : 0;
+            cp_async_16(dst + j * 1024,
+                        vb ? a.kv + static_cast<size_t>(row) * a.d_kv + c * 64 + c16 * 8 : a.kv,
+                        vb * 2);
           }
         }
+        cp_async_commit();
       }
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      mbar_arrive(&tile_full[b]);
+      for (int c = 0; c < nc; ++c) {
+        cp_async_wait_dyn(nc - 1 - c);  // groups 0..c have landed
+        fence_proxy_async_smem();
+        mbar_arrive(&chunk_full[c]);
+      }
     }
     cp_async_wait<0>();
   } else if (warp == 5 + kProducers) {
@@ -207,11 +234,12 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       // ---------------------------------------------------------------- query-chunk TMA
       prefetch_tmap(&qmap);
       int qn = 0;
-      for (int i = 0; i < n_tiles; ++i)
+      const int n_pairs = (n_tiles + 1) / 2;  // one pass over the query per pair of tiles
+      for (int g = 0; g < n_pairs; ++g)
         for (int c = 0; c < nc; ++c, ++qn) {
           const int slot = qn % kQRing;
           if (!mbar_wait(&q_empty[slot], ((qn / kQRing) & 1) ^ 1, abort_flag, 41)) {
-            i = n_tiles;
+            g = n_pairs;
             break;
           }
           if (a.inject && blockIdx.x == 0 && blockIdx.y == 0 && qn == 0) continue;
@@ -251,14 +279,17 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
         mma_commit(pv_done);
         return true;
       };
-      for (int i = 0; ok && i < n_tiles; ++i) {
-        const int st = i & 1;
-        if (!mbar_wait(&s_free[st], ((i >> 1) & 1) ^ 1, abort_flag, 43)) break;
-        if (!mbar_wait(&tile_full[st], (i >> 1) & 1, abort_flag, 46)) break;
-        const uint32_t tb = tile_base + st * kTile;
+      // Tiles go in pairs: one pass over the query chunks computes the scores of both
+      // (S buffers 0 and 1), then P.V of each as its softmax is ready.
+      for (int g = 0; ok && 2 * g < n_tiles; ++g) {
+        const int ia = 2 * g;
+        const bool has_b = ia + 1 < n_tiles;
+        if (!mbar_wait(&s_free[0], (g & 1) ^ 1, abort_flag, 43)) break;
+        if (has_b && !mbar_wait(&s_free[1], (g & 1) ^ 1, abort_flag, 43)) break;
         for (int c = 0; c < nc; ++c, ++qn) {
           const int slot = qn % kQRing;
-          if (!mbar_wait(&q_full[slot], (qn / kQRing) & 1, abort_flag, 44)) {
+          if (!mbar_wait(&chunk_full[c], g & 1, abort_flag, 46) ||
+              !mbar_wait(&q_full[slot], (qn / kQRing) & 1, abort_flag, 44)) {
             ok = false;
             break;
           }
@@ -266,20 +297,26 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
           fence_proxy_async_smem();
           const uint32_t qb = q_base + slot * kQChunk;
           const int w = min(64, a.d_kv - c * 64);
-          for (int ks = 0; ks < (w + 15) / 16; ++ks)
-            mma_bf16(tmem + st * kBN, smem_desc(qb + ks * 32, 16, 1024, kSw128),
-                     smem_desc(tb + c * kKVChunk + ks * 32, 16, 1024, kSw128), idesc_s,
-                     (c > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < (w + 15) / 16; ++ks) {
+            const uint64_t qd = smem_desc(qb + ks * 32, 16, 1024, kSw128);
+            const uint32_t acc = (c > 0 || ks > 0) ? 1u : 0u;
+            mma_bf16(tmem, qd, smem_desc(tile_base + c * kKVChunk + ks * 32, 16, 1024, kSw128),
+                     idesc_s, acc);
+            if (has_b)
+              mma_bf16(tmem + kBN, qd,
+                       smem_desc(tile_base + kTile + c * kKVChunk + ks * 32, 16, 1024, kSw128),
+                       idesc_s, acc);
+          }
           mma_commit(&q_empty[slot]);
         }
         if (!ok) break;
-        mma_commit(&s_full[st]);
-        if (i > 0 && !do_pv(i - 1)) {
+        mma_commit(&s_full[0]);
+        if (has_b) mma_commit(&s_full[1]);
+        if (!do_pv(ia) || (has_b && !do_pv(ia + 1))) {
           ok = false;
           break;
         }
       }
-      if (ok && n_tiles > 0) do_pv(n_tiles - 1);
       mma_commit(drain);
       mbar_wait_drain(drain, 0);
     }
@@ -400,7 +437,12 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
       }
       if (vg == 0 && h < a.H && a.lse) a.lse[static_cast<size_t>(t) * a.H + h] = lse_val;
     } else {
+      // Each thread stages its head row (nvg * 64 fp32) in the tile buffers, now idle, and
+      // sends it with one bulk store.  Staged rows are 16 bytes longer than the data, so
+      // the rows of a warp start in different bank groups.
       const size_t row = (static_cast<size_t>(t) * a.splits + split) * a.H + h;
+      const int n16 = a.nvg * 8;  // 16-byte pieces per row (fp16)
+      uint4* srow = reinterpret_cast<uint4*>(tiles + static_cast<size_t>(h) * (n16 + 1) * 16);
       for (int c = 0; c < a.nvg * 64; c += 32) {
         float o[32];
         if (have) {  // warp-uniform
@@ -410,15 +452,24 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = 0.f;
         }
-        if (h < a.H) {
-          float4* dst = reinterpret_cast<float4*>(a.part_o + row * a.d_v + vbase + c);
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(o[4 * j] * inv_l, o[4 * j + 1] * inv_l, o[4 * j + 2] * inv_l,
-                                 o[4 * j + 3] * inv_l);
+        for (int j = 0; j < 4; ++j) {
+          uint32_t hv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __half2 h2 = __floats2half2_rn(o[8 * j + 2 * e] * inv_l, o[8 * j + 2 * e + 1] * inv_l);
+            hv[e] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          srow[c / 8 + j] = make_uint4(hv[0], hv[1], hv[2], hv[3]);
         }
       }
-      if (vg == 0 && h < a.H) a.part_lse[row] = lse_val;
+      fence_proxy_async_smem();
+      if (h < a.H) {
+        bulk_store(a.part_o + row * a.d_v + vbase, srow, n16 * 16);
+        bulk_commit();
+        if (vg == 0) a.part_lse[row] = lse_val;
+        bulk_wait_read();
+      }
     }
   }
 
@@ -431,59 +482,64 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
 }
 
 // Merge split-KV partial results: O = sum_s exp(lse_s - LSE) O_s, LSE = logsumexp_s lse_s.
-__global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restrict__ part_o,
+// Every thread reads the split LSEs itself (the same few words for the whole CTA) beside
+// its 4 dims of each partial, kBatch splits at a time with all loads issued together, and
+// folds each batch in under a running maximum: no shared memory, no block barrier.
+__global__ void __launch_bounds__(128) attn_combine_kernel(const uint16_t* __restrict__ part_o,
                                                            const float* __restrict__ part_lse,
                                                            int splits, int H, int d_v,
                                                            uint16_t* __restrict__ out,
                                                            float* __restrict__ lse) {
   const int t = blockIdx.y, h = blockIdx.x;
-  __shared__ float wsh[64];
-  __shared__ float lse_sh;
-  if (threadIdx.x < 32) {
-    float m = -INFINITY;
-    for (int s = threadIdx.x; s < splits; s += 32)
-      m = fmaxf(m, part_lse[(static_cast<size_t>(t) * splits + s) * H + h]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float sum = 0.f;
-    for (int s = threadIdx.x; s < splits; s += 32) {
-      const float ls = part_lse[(static_cast<size_t>(t) * splits + s) * H + h];
-      const float e = (m == -INFINITY || ls == -INFINITY) ? 0.f : __expf(ls - m);
-      wsh[s] = e;
-      sum += e;
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float inv = sum > 0.f ? 1.f / sum : 0.f;
-    for (int s = threadIdx.x; s < splits; s += 32) wsh[s] *= inv;
-    if (threadIdx.x == 0) lse_sh = sum > 0.f ? m + __logf(sum) : -INFINITY;
-  }
-  __syncthreads();
+  const float* pls = part_lse + static_cast<size_t>(t) * splits * H + h;  // split s: pls[s * H]
+  const uint16_t* po = part_o + (static_cast<size_t>(t) * splits * H + h) * d_v;
   for (int d = threadIdx.x * 4; d < d_v; d += blockDim.x * 4) {
-    // every split's partial is loaded before the sum (independent loads, one round trip)
+    float m = -INFINITY, sum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     constexpr int kBatch = 16;
     for (int s0 = 0; s0 < splits; s0 += kBatch) {
+      float ls[kBatch];
       float4 v[kBatch];
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u)
-        v[u] = s0 + u < splits ? *reinterpret_cast<const float4*>(
-                                     part_o + ((static_cast<size_t>(t) * splits + s0 + u) * H + h) *
-                                                  d_v + d)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < kBatch; ++u) {
+        const bool in = s0 + u < splits;
+        ls[u] = in ? pls[static_cast<size_t>(s0 + u) * H] : -INFINITY;
+        if (in) {
+          const uint2 raw =
+              *reinterpret_cast<const uint2*>(po + static_cast<size_t>(s0 + u) * H * d_v + d);
+          const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+          const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+          v[u] = make_float4(lo.x, lo.y, hi.x, hi.y);
+        } else {
+          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      float mb = m;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) mb = fmaxf(mb, ls[u]);
+      if (mb == -INFINITY) continue;
+      const float sc = m == -INFINITY ? 0.f : __expf(m - mb);
+      acc.x *= sc;
+      acc.y *= sc;
+      acc.z *= sc;
+      acc.w *= sc;
+      sum *= sc;
+      m = mb;
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
-        const float w = s0 + u < splits ? wsh[s0 + u] : 0.f;
-        acc.x = fmaf(w, v[u].x, acc.x);
-        acc.y = fmaf(w, v[u].y, acc.y);
-        acc.z = fmaf(w, v[u].z, acc.z);
-        acc.w = fmaf(w, v[u].w, acc.w);
+        const float e = ls[u] == -INFINITY ? 0.f : __expf(ls[u] - m);
+        sum += e;
+        acc.x = fmaf(e, v[u].x, acc.x);
+        acc.y = fmaf(e, v[u].y, acc.y);
+        acc.z = fmaf(e, v[u].z, acc.z);
+        acc.w = fmaf(e, v[u].w, acc.w);
       }
     }
-    uint2 pk = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
+    uint2 pk = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
     *reinterpret_cast<uint2*>(out + (static_cast<size_t>(t) * H + h) * d_v + d) = pk;
+    if (d == 0 && lse) lse[static_cast<size_t>(t) * H + h] = sum > 0.f ? m + __logf(sum) : -INFINITY;
   }
-  if (threadIdx.x == 0 && lse) lse[static_cast<size_t>(t) * H + h] = lse_sh;
 }
 
 // ---------------------------------------------------------------------------- host
@@ -503,7 +559,7 @@ size_t attn_ws_bytes(int32_t T, int32_t H, int32_t d_v, int32_t k) {
   if (T <= 0) return 0;
   const int splits = attn_splits(T, k, attn_groups(d_v));
   if (splits <= 1) return 0;
-  const size_t o = static_cast<size_t>(T) * splits * H * d_v * 4;
+  const size_t o = static_cast<size_t>(T) * splits * H * d_v * 2;
   const size_t l = static_cast<size_t>(T) * splits * H * 4;
   return ((o + 255) & ~static_cast<size_t>(255)) + ((l + 255) & ~static_cast<size_t>(255));
 }
@@ -579,8 +635,8 @@ cudaError_t launch_attn(const AttnLaunch& L) {
   a.part_lse = nullptr;
   a.inject = take_injection(2);
   if (splits > 1) {
-    const size_t o = static_cast<size_t>(T) * splits * L.n_heads * L.d_v * 4;
-    a.part_o = static_cast<float*>(L.ws);
+    const size_t o = static_cast<size_t>(T) * splits * L.n_heads * L.d_v * 2;
+    a.part_o = static_cast<uint16_t*>(L.ws);
     a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(L.ws) +
                                           ((o + 255) & ~static_cast<size_t>(255)));
   }
