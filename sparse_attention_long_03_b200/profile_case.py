@@ -1,0 +1,80 @@
+"""Run one synthetic workload through one stage of the DSA path a fixed number of times,
+for an external profiler (launch lists, hardware counters).  Nothing is timed here and
+nothing is checked: the device buffers are built once, then W + N launches run back to
+back on one stream.
+
+    python -m sparse_attention_long_03_b200.profile_case WORKLOAD STAGE [--warmup W] [--launches N]
+
+STAGE is one of: forward (dsa_forward), indexer (dsa_indexer_logits), topk (dsa_topk on
+the indexer's logits), attention (dsa_sparse_mla_attn on the forward's selection).
+"""
+
+from __future__ import annotations
+
+import argparse
+
+import numpy as np
+import torch
+
+from . import dsa
+from . import workloads as W
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("workload", choices=sorted(W.CONFIGS))
+    ap.add_argument("stage", choices=["forward", "indexer", "topk", "attention"])
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--launches", type=int, default=1)
+    args = ap.parse_args(argv)
+
+    dev = torch.device("cuda", 0)
+    cfg, cache, qs = W.make(args.workload)
+    T, H = qs.n_tokens, cfg.n_heads
+    max_pos = int(qs.tok_pos.max())
+    k8 = torch.from_numpy(cache.k8).to(dev)
+    ks = torch.from_numpy(cache.k_scale).to(dev)
+    kv = torch.from_numpy(cache.kv.view(np.int16)).to(dev)
+    bt = torch.from_numpy(cache.block_table).to(dev)
+    c = dsa.make_cache(k8, ks, kv, bt)
+    tok_seq = torch.from_numpy(qs.tok_seq).to(dev)
+    tok_pos = torch.from_numpy(qs.tok_pos).to(dev)
+    queries = dsa.make_queries(tok_seq, tok_pos, max_pos)
+    q8 = torch.from_numpy(qs.q8).to(dev)
+    q_scale = torch.from_numpy(qs.q_scale).to(dev)
+    w = torch.from_numpy(qs.w).to(dev)
+    q = torch.from_numpy(qs.q.view(np.int16)).to(dev)
+    out = torch.zeros((T, H, cfg.d_v), dtype=torch.int16, device=dev)
+    lse = torch.zeros((T, H), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, cfg.topk), dtype=torch.int32, device=dev)
+    logits = torch.empty((T, ((max_pos + 1 + 127) // 128) * 128), dtype=torch.float32,
+                         device=dev)
+    ws = torch.empty(dsa.forward_workspace_size(T, max_pos, cfg.topk, H, cfg.d_v),
+                     dtype=torch.uint8, device=dev)
+
+    def forward():
+        dsa.dsa_forward(c, queries, q8, q_scale, w, q, cfg.d_v, cfg.scale, cfg.topk, out, lse,
+                        idx, ws)
+
+    run = {
+        "forward": forward,
+        "indexer": lambda: dsa.dsa_indexer_logits(c, queries, q8, q_scale, w, logits),
+        "topk": lambda: dsa.dsa_topk(logits, queries, cfg.topk, idx),
+        "attention": lambda: dsa.dsa_sparse_mla_attn(c, queries, q, cfg.d_v, cfg.scale, idx,
+                                                     out, lse),
+    }[args.stage]
+    if args.stage == "topk":
+        dsa.dsa_indexer_logits(c, queries, q8, q_scale, w, logits)
+    if args.stage == "attention":
+        forward()
+    for _ in range(args.warmup + args.launches):
+        run()
+    torch.cuda.synchronize()
+    status = dsa.dsa_read_device_status()
+    print(f"{args.workload} {args.stage}: {args.warmup} + {args.launches} launches, "
+          f"device status {status}")
+    return 0 if status == 0 else 1
+
+
+if __name__ == "__main__":
+    raise SystemExit(main())
