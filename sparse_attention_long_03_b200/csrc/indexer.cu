@@ -203,6 +203,8 @@ constexpr int kIdxThreads = (3 + kEpiWarps) * 32;
 // so with eleven warps three schedulers hold three: bound registers as for twelve warps.
 constexpr int kIdxThreadsBound = 12 * 32;
 // Key tiles the producer warp issues per pass (one per lane), at most.
+// Work-balance weight of a run, in key tiles (staging its query, handing over its slot).
+constexpr int kRunCost = 8;
 constexpr int kProducerBatch = 4;
 
 __host__ __device__ constexpr int pow2ceil(int x) {
@@ -363,8 +365,26 @@ __global__ void __launch_bounds__(kIdxThreadsBound, 1)
     pv = plan_view(inline_plan ? static_cast<void*>(splan) : a.plan, a.T);
     const int n_runs = pv.hdr[0];
     const int total = pv.hdr[1];
-    i0 = static_cast<int>(static_cast<int64_t>(total) * blockIdx.x / gridDim.x);
-    i1 = static_cast<int>(static_cast<int64_t>(total) * (blockIdx.x + 1) / gridDim.x);
+    // Slices are equal in work, not in tiles: a run costs kRunCost tiles on top of its
+    // own (its query is staged and its slot handed over), so CTAs whose slice crosses many
+    // short runs get fewer tiles.  Position u of the weighted list lies in run r, the last
+    // with item0[r] + kRunCost * r <= u; it maps to the tile min(u - that, tiles of r) of
+    // the run (a position in a run's overhead maps to the next run's first tile).
+    const int64_t wtot = static_cast<int64_t>(total) + static_cast<int64_t>(kRunCost) * n_runs;
+    auto item_at = [&](int64_t u) -> int {
+      if (n_runs <= 0) return 0;
+      int rlo = 0, rhi = n_runs;
+      while (rhi - rlo > 1) {
+        const int mid = (rlo + rhi) >> 1;
+        if (pv.item0[mid] + static_cast<int64_t>(kRunCost) * mid <= u) rlo = mid;
+        else rhi = mid;
+      }
+      const int64_t off = u - (pv.item0[rlo] + static_cast<int64_t>(kRunCost) * rlo);
+      const int len = pv.item0[rlo + 1] - pv.item0[rlo];
+      return pv.item0[rlo] + static_cast<int>(off < len ? off : len);
+    };
+    i0 = item_at(wtot * blockIdx.x / gridDim.x);
+    i1 = item_at(wtot * (blockIdx.x + 1) / gridDim.x);
     lo = 0;
     int hi = n_runs;  // item0[lo] <= i0 < item0[hi]
     while (i0 < i1 && hi - lo > 1) {

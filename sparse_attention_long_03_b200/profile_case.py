@@ -1,12 +1,16 @@
 """Run one synthetic workload through one stage of the DSA path a fixed number of times,
-for an external profiler (launch lists, hardware counters).  Nothing is timed here and
-nothing is checked: the device buffers are built once, then W + N launches run back to
-back on one stream.
+for an external profiler (launch lists, hardware counters), or timed with --time.  Nothing
+is checked: the device buffers are built once, then W + N launches run back to back on one
+stream.
 
     python -m sparse_attention_long_03_b200.profile_case WORKLOAD STAGE [--warmup W] [--launches N]
 
 STAGE is one of: forward (dsa_forward), indexer (dsa_indexer_logits), topk (dsa_topk on
 the indexer's logits), attention (dsa_sparse_mla_attn on the forward's selection).
+
+With --time the N launches after the warm-up are timed with CUDA events on the launching
+stream and the mean per launch is printed (for the indexer also its FP8 work rate: every
+causal (query token, key) pair costs heads x idx_dim multiply-adds).
 """
 
 from __future__ import annotations
@@ -26,6 +30,7 @@ def main(argv=None):
     ap.add_argument("stage", choices=["forward", "indexer", "topk", "attention"])
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--launches", type=int, default=1)
+    ap.add_argument("--time", action="store_true")
     args = ap.parse_args(argv)
 
     dev = torch.device("cuda", 0)
@@ -67,12 +72,29 @@ def main(argv=None):
         dsa.dsa_indexer_logits(c, queries, q8, q_scale, w, logits)
     if args.stage == "attention":
         forward()
-    for _ in range(args.warmup + args.launches):
+    for _ in range(args.warmup):
         run()
     torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.launches):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
     status = dsa.dsa_read_device_status()
-    print(f"{args.workload} {args.stage}: {args.warmup} + {args.launches} launches, "
-          f"device status {status}")
+    line = (f"{args.workload} {args.stage}: {args.warmup} + {args.launches} launches, "
+            f"device status {status}")
+    if args.time:
+        us = e0.elapsed_time(e1) * 1000.0 / max(1, args.launches)
+        line += f"; {us:.1f} us per launch ({T} query tokens)"
+        if args.stage == "indexer":
+            pairs = int((qs.tok_pos.astype(np.int64) + 1).sum())
+            flop = 2.0 * pairs * cfg.n_idx_heads * cfg.idx_dim
+            line += f"; {flop / (us * 1e-6) / 1e12:.1f} TFLOP/s FP8 ({flop:.3e} FLOP)"
+        if args.stage == "forward":
+            line += f"; {T / (us * 1e-6):.0f} query tokens/s"
+    print(line)
     return 0 if status == 0 else 1
 
 
