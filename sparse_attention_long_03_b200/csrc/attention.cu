@@ -165,6 +165,11 @@ __global__ void __launch_bounds__(attn::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tmem_o = tmem + 2 * kBN;
+  // Launched as a programmatic dependent of the top-k: everything above ran while it
+  // finished.  The selection (and the slots this grid writes) need its completion; the
+  // query-chunk warp reads only the query, an input, and starts streaming at once.
+  pdl_trigger();
+  if (warp != 5 + kProducers) pdl_wait();
 
   if (warp >= 5 && warp < 5 + kProducers) {
     // ---------------------------------------------------------------- gatherers (2 warps)
@@ -490,6 +495,8 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const uint16_t* __res
                                                            int splits, int H, int d_v,
                                                            uint16_t* __restrict__ out,
                                                            float* __restrict__ lse) {
+  pdl_wait();  // the partials come from the attention kernel
+  pdl_trigger();
   const int t = blockIdx.y, h = blockIdx.x;
   const float* pls = part_lse + static_cast<size_t>(t) * splits * H + h;  // split s: pls[s * H]
   const uint16_t* po = part_o + (static_cast<size_t>(t) * splits * H + h) * d_v;
@@ -640,15 +647,12 @@ cudaError_t launch_attn(const AttnLaunch& L) {
     a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(L.ws) +
                                           ((o + 255) & ~static_cast<size_t>(255)));
   }
-  sparse_mla_kernel<<<dim3(groups * splits, T), attn::kThreads, attn::kSmemAlloc, L.stream>>>(qmap,
-                                                                                           a);
-  count_launch();
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(sparse_mla_kernel, dim3(groups * splits, T), dim3(attn::kThreads),
+                             attn::kSmemAlloc, L.stream, qmap, a);
   if (e != cudaSuccess || splits == 1) return e;
-  attn_combine_kernel<<<dim3(L.n_heads, T), 128, 0, L.stream>>>(a.part_o, a.part_lse, splits,
-                                                                L.n_heads, L.d_v, L.out, L.lse);
-  count_launch();
-  return cudaGetLastError();
+  return launch_pdl(attn_combine_kernel, dim3(L.n_heads, T), dim3(128), 0, L.stream,
+                    static_cast<const uint16_t*>(a.part_o), static_cast<const float*>(a.part_lse),
+                    splits, L.n_heads, L.d_v, L.out, L.lse);
 }
 
 }  // namespace dsa
