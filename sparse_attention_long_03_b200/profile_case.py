@@ -34,12 +34,13 @@ def main(argv=None):
     args = ap.parse_args(argv)
 
     dev = torch.device("cuda", 0)
-    cfg, cache, qs = W.make(args.workload)
+    need_kv = args.stage in ("forward", "attention")
+    cfg, cache, qs = W.make(args.workload, with_kv=need_kv, with_q=need_kv)
     T, H = qs.n_tokens, cfg.n_heads
     max_pos = int(qs.tok_pos.max())
     k8 = torch.from_numpy(cache.k8).to(dev)
     ks = torch.from_numpy(cache.k_scale).to(dev)
-    kv = torch.from_numpy(cache.kv.view(np.int16)).to(dev)
+    kv = torch.from_numpy(cache.kv.view(np.int16)).to(dev) if need_kv else None
     bt = torch.from_numpy(cache.block_table).to(dev)
     c = dsa.make_cache(k8, ks, kv, bt)
     tok_seq = torch.from_numpy(qs.tok_seq).to(dev)
@@ -48,14 +49,18 @@ def main(argv=None):
     q8 = torch.from_numpy(qs.q8).to(dev)
     q_scale = torch.from_numpy(qs.q_scale).to(dev)
     w = torch.from_numpy(qs.w).to(dev)
-    q = torch.from_numpy(qs.q.view(np.int16)).to(dev)
-    out = torch.zeros((T, H, cfg.d_v), dtype=torch.int16, device=dev)
-    lse = torch.zeros((T, H), dtype=torch.float32, device=dev)
     idx = torch.empty((T, cfg.topk), dtype=torch.int32, device=dev)
-    logits = torch.empty((T, ((max_pos + 1 + 127) // 128) * 128), dtype=torch.float32,
-                         device=dev)
-    ws = torch.empty(dsa.forward_workspace_size(T, max_pos, cfg.topk, H, cfg.d_v),
-                     dtype=torch.uint8, device=dev)
+    # only the buffers the stage touches are allocated (prefill ones are gigabytes)
+    q = out = lse = ws = logits = None
+    if need_kv:
+        q = torch.from_numpy(qs.q.view(np.int16)).to(dev)
+        out = torch.zeros((T, H, cfg.d_v), dtype=torch.int16, device=dev)
+        lse = torch.zeros((T, H), dtype=torch.float32, device=dev)
+        ws = torch.empty(dsa.forward_workspace_size(T, max_pos, cfg.topk, H, cfg.d_v),
+                         dtype=torch.uint8, device=dev)
+    else:
+        logits = torch.empty((T, ((max_pos + 1 + 127) // 128) * 128), dtype=torch.float32,
+                             device=dev)
 
     def forward():
         dsa.dsa_forward(c, queries, q8, q_scale, w, q, cfg.d_v, cfg.scale, cfg.topk, out, lse,
