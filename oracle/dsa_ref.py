@@ -20,12 +20,17 @@ selection -> sparse core attention") and its Spanish translation
       every query head h attends to the same 576-wide latent rows, whose first 512
       values are the value vector.
 
-Readings of points the pages leave open (each one is listed in the design doc):
+Readings of points the pages leave open:
   * causality includes the token itself: s ranges over [0, pos(t)];
   * ties in (2) go to the smaller position s; fewer than k valid keys -> all of them;
   * FP8 is e4m3 "fn" (bias 7, no infinities, S.1111.111 = NaN, max 448), one fp32
     scale per token; BF16 is the upper half of an IEEE fp32;
-  * the softmax uses max subtraction and returns LSE = max + log(sum exp).
+  * the softmax uses max subtraction and returns LSE = max + log(sum exp);
+  * appending a token to the caches (the step before the path: the pages' paginated
+    caches, "Open kernels" on "DeepSeek V3.2-Exp: Sparse Attention, Long Context, and
+    Cheaper API") quantises its index key with scale = amax / 448 (1 if amax = 0) and
+    codes = e4m3(key / scale), round to nearest even, saturating; the division and the
+    rounding decision are taken in fp32, as the kernel takes them.
 
 Every function below is pinned by tests/test_oracle_pins.py (closed forms,
 brute force on tiny inputs, library special cases and invariants).
@@ -58,6 +63,39 @@ def decode_e4m3(b) -> np.ndarray:
     return np.where((e == 0xF) & (m == 0x7), np.nan, val)
 
 
+E4M3_MAX = 448.0
+
+
+def encode_e4m3(v) -> np.ndarray:
+    """float32 values -> e4m3 ("fn") bytes: the nearest finite e4m3 value, a tie going to
+    the even code (even mantissa), magnitudes beyond 448 saturating to 448; NaN -> 0x7F
+    with the sign; the sign of zero is kept.
+
+    Built from the value table of the positive codes 0x00..0x7E (monotone in the code).
+    """
+    v = np.asarray(v, dtype=np.float32).astype(np.float64)  # exact widening
+    table = decode_e4m3(np.arange(0x7F, dtype=np.uint8))    # 0, 2^-9, ..., 448
+    a = np.abs(v)
+    sat = np.minimum(np.nan_to_num(a, nan=0.0), E4M3_MAX)
+    hi = np.clip(np.searchsorted(table, sat, side="left"), 0, 0x7E)  # table[hi] >= sat
+    lo = np.maximum(hi - 1, 0)
+    d_lo = sat - table[lo]
+    d_hi = table[hi] - sat
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    code = np.where(np.isnan(v), np.uint8(0x7F), code)
+    return (code | np.where(np.signbit(v), np.uint8(0x80), np.uint8(0))).astype(np.uint8)
+
+
+def quantize_key(x):
+    """One token's index key (fp32 [D]) -> (e4m3 codes uint8 [D], fp32 scale):
+    scale = amax / 448 in fp32 (1 if amax = 0), codes = encode_e4m3(fp32(x / scale))."""
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(x))) if x.size else np.float32(0.0)
+    scale = np.float32(amax / np.float32(E4M3_MAX)) if amax > 0 else np.float32(1.0)
+    return encode_e4m3((x / scale).astype(np.float32)), scale
+
+
 def decode_bf16(u) -> np.ndarray:
     """BF16 bit patterns (uint16) -> float64: they are the upper 16 bits of an fp32."""
     u = np.asarray(u, dtype=np.uint16).astype(np.uint32) << 16
@@ -76,6 +114,39 @@ def logical_rows(block_table, b: int, n: int, page: int = PAGE) -> np.ndarray:
     """
     s = np.arange(n, dtype=np.int64)
     return np.asarray(block_table)[b, s // page].astype(np.int64) * page + s % page
+
+
+def cache_append(k8, k_scale, kv, block_table, tok_seq, tok_pos, k_in, kv_in,
+                 page: int = PAGE):
+    """Append new tokens to the paged caches; returns (k8, k_scale, kv, ok) as new arrays.
+
+    Token i of sequence tok_seq[i] at position tok_pos[i] lands in the physical row
+    block_table[seq][pos // page] * page + pos % page: its index key k_in[i] (fp32) is
+    quantised by quantize_key, its latent row kv_in[i] (bf16 bit patterns) copied.  A token
+    whose sequence, position or block-table entry is out of range is not written
+    (ok[i] = False).  kv / kv_in may be None (index keys only).
+    """
+    k8 = np.array(k8, dtype=np.uint8, copy=True)
+    k_scale = np.array(k_scale, dtype=np.float32, copy=True)
+    kv = None if kv is None else np.array(kv, dtype=np.uint16, copy=True)
+    bt = np.asarray(block_table)
+    n_rows = k8.shape[0]
+    ok = np.zeros(len(tok_seq), dtype=bool)
+    for i, (b, p) in enumerate(zip(tok_seq, tok_pos)):
+        b, p = int(b), int(p)
+        if not (0 <= b < bt.shape[0] and 0 <= p < bt.shape[1] * page):
+            continue
+        blk = int(bt[b, p // page])
+        if not (0 <= blk < n_rows // page):
+            continue
+        row = blk * page + p % page
+        codes, sc = quantize_key(k_in[i])
+        k8[row] = codes
+        k_scale[row] = sc
+        if kv is not None and kv_in is not None:
+            kv[row] = np.asarray(kv_in[i], dtype=np.uint16)
+        ok[i] = True
+    return k8, k_scale, kv, ok
 
 
 # --------------------------------------------------------------------------------------
