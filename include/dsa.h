@@ -147,6 +147,33 @@ DSA_API dsa_status dsa_forward(const dsa_paged_cache* cache, const dsa_queries* 
 DSA_API size_t dsa_forward_workspace_size(int32_t n_tokens, int32_t max_pos, int32_t k,
                                   int32_t n_heads, int32_t d_v);
 
+/* (0) Cache append: write n_new new tokens into the paged caches the path reads (the
+ * pages' paginated caches with 64-token pages: "DeepSeek V3.2-Exp: Sparse Attention, Long
+ * Context, and Cheaper API", sections "Quick guide to run it locally" and "Open kernels";
+ * FP8 index keys: "DeepSeek V3.2-Exp Cuts Prolonged-Context Costs ...", section "FP8 index
+ * -> top-k selection -> sparse core attention").  Token i of sequence tok_seq[i] at position
+ * tok_pos[i] goes to the physical row r = block_table[b * max_blocks_per_seq + pos / 64] * 64
+ * + pos % 64 (geometry and block table from `cache`):
+ *   k_scale[r]       = s = max_d |k_in[i, d]| / 448 in fp32 (s = 1 if that maximum is 0)
+ *   k8[r, 0:idx_dim] = e4m3(k_in[i, :] / s): fp32 division, round to nearest even,
+ *                      magnitudes beyond 448 saturating to 448
+ *   kv[r, 0:d_kv]    = kv_in[i, :] copied (skipped when kv or kv_in is NULL)
+ * k8, k_scale, kv  device caches, written (normally the buffers `cache` describes; its
+ *                  own pointers are not used)
+ * tok_seq, tok_pos device int32 [n_new]
+ * k_in             device fp32 [n_new, idx_dim], row-major
+ * kv_in            device bf16 [n_new, d_kv], row-major, or NULL
+ * New tokens must name distinct rows (two tokens with one row race).  A token whose
+ * sequence, position or block-table entry is out of range is skipped and recorded
+ * (DSA_ERR_BAD_INDEX through dsa_read_device_status).  Host checks: NULL k8 / k_scale /
+ * tok_seq / tok_pos / k_in, n_new < 0, idx_dim not a multiple of 4 or above 1024, d_kv not
+ * a multiple of 8 -> DSA_ERR_INVALID_ARG; page_size other than 64 -> DSA_ERR_UNSUPPORTED.
+ * Asynchronous on `stream`; allocates nothing.                                           */
+DSA_API dsa_status dsa_cache_append(const dsa_paged_cache* cache, uint8_t* k8, float* k_scale,
+                                    uint16_t* kv, int32_t n_new, const int32_t* tok_seq,
+                                    const int32_t* tok_pos, const float* k_in,
+                                    const uint16_t* kv_in, void* stream);
+
 /* Waits for `stream`, then returns and clears the device status word of the current
  * device (DSA_OK, DSA_ERR_BAD_INDEX or DSA_ERR_TIMEOUT; DSA_ERR_CUDA if the wait failed). */
 DSA_API dsa_status dsa_read_device_status(void* stream);

@@ -145,6 +145,28 @@ int64_t dsa_launch_count(void) { return g_launches.load(); }
 
 uint32_t dsa_debug_timeout_site(void) { return g_last_where; }
 
+dsa_status dsa_cache_append(const dsa_paged_cache* cache, uint8_t* k8, float* k_scale,
+                            uint16_t* kv, int32_t n_new, const int32_t* tok_seq,
+                            const int32_t* tok_pos, const float* k_in, const uint16_t* kv_in,
+                            void* stream) {
+  using namespace dsa;
+  if (!cache || !cache->block_table || n_new < 0) return DSA_ERR_INVALID_ARG;
+  if (cache->batch <= 0 || cache->max_blocks_per_seq <= 0 || cache->num_blocks <= 0)
+    return DSA_ERR_INVALID_ARG;
+  if (cache->page_size != kPage) return DSA_ERR_UNSUPPORTED;
+  if (cache->idx_dim <= 0 || cache->idx_dim % 4 || cache->idx_dim > 1024)
+    return DSA_ERR_INVALID_ARG;
+  if (n_new == 0) return DSA_OK;
+  if (!k8 || !k_scale || !tok_seq || !tok_pos || !k_in) return DSA_ERR_INVALID_ARG;
+  if (!aligned(k8, 4) || !aligned(k_scale, 4) || !aligned(k_in, 16)) return DSA_ERR_INVALID_ARG;
+  const bool copy_kv = kv && kv_in;
+  if (copy_kv && (cache->d_kv <= 0 || cache->d_kv % 8 || !aligned(kv, 16) || !aligned(kv_in, 16)))
+    return DSA_ERR_INVALID_ARG;
+  return cuda_status(launch_cache_append(cache, k8, k_scale, copy_kv ? kv : nullptr, n_new,
+                                         tok_seq, tok_pos, k_in, copy_kv ? kv_in : nullptr,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 int32_t dsa_last_cuda_error(void) { return g_last_cuda_error.load(); }
 
 dsa_status dsa_debug_inject(int32_t fault) {

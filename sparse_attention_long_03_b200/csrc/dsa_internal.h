@@ -40,6 +40,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return e;
 }
 
+// ---- cache append -------------------------------------------------------------------
+cudaError_t launch_cache_append(const dsa_paged_cache* c, uint8_t* k8, float* k_scale,
+                                uint16_t* kv, int32_t n_new, const int32_t* tok_seq,
+                                const int32_t* tok_pos, const float* k_in, const uint16_t* kv_in,
+                                cudaStream_t stream);
+
 // ---- indexer ------------------------------------------------------------------------
 size_t indexer_ws_bytes(int32_t n_tokens);
 struct IndexerLaunch {

@@ -29,7 +29,7 @@ EXPORTED = ("dsa_indexer_logits", "dsa_indexer_workspace_size", "dsa_indexer_log
             "dsa_topk_workspace_size", "dsa_sparse_mla_attn", "dsa_attn_workspace_size",
             "dsa_forward", "dsa_forward_workspace_size", "dsa_read_device_status",
             "dsa_launch_count", "dsa_status_string", "dsa_abi_version", "dsa_debug_inject",
-            "dsa_debug_timeout_site", "dsa_last_cuda_error")
+            "dsa_debug_timeout_site", "dsa_last_cuda_error", "dsa_cache_append")
 
 
 class DsaError(RuntimeError):
@@ -93,6 +93,7 @@ def lib() -> ctypes.CDLL:
             "dsa_debug_inject": (I32, [I32]),
             "dsa_debug_timeout_site": (ctypes.c_uint32, []),
             "dsa_last_cuda_error": (I32, []),
+            "dsa_cache_append": (I32, [PC, P, P, P, I32, P, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -128,14 +129,18 @@ def make_cache(k8: torch.Tensor, k_scale: torch.Tensor, kv: Optional[torch.Tenso
     """Describe device caches: k8 uint8 [rows, D_I], k_scale fp32 [rows],
     kv uint16/int16/bf16 [rows, D_kv], block_table int32 [B, max_blocks]."""
     rows = k8.shape[0] if k8 is not None else kv.shape[0]
-    return PagedCache(
+    c = PagedCache(
         _ptr(k8), _ptr(k_scale), _ptr(kv), _ptr(block_table), block_table.shape[0],
         block_table.shape[1], rows // page_size, page_size,
         k8.shape[1] if k8 is not None else 0, kv.shape[1] if kv is not None else 0)
+    c._tensors = (k8, k_scale, kv, block_table)  # the struct holds raw pointers into these
+    return c
 
 
 def make_queries(tok_seq: torch.Tensor, tok_pos: torch.Tensor, max_pos: int) -> Queries:
-    return Queries(tok_seq.shape[0], _ptr(tok_seq), _ptr(tok_pos), int(max_pos))
+    q = Queries(tok_seq.shape[0], _ptr(tok_seq), _ptr(tok_pos), int(max_pos))
+    q._tensors = (tok_seq, tok_pos)  # the struct holds raw pointers into these
+    return q
 
 
 def _workspace(nbytes: int, device) -> torch.Tensor:
@@ -216,6 +221,17 @@ def dsa_forward(cache: PagedCache, queries: Queries, q8, q_scale, w, q, d_v: int
                            _stream(stream))
     _check("dsa_forward", st)
     return out
+
+
+def dsa_cache_append(cache: PagedCache, k8, k_scale, kv, tok_seq, tok_pos, k_in, kv_in=None,
+                     stream=None):
+    """(0) Write new tokens into the paged caches: k8[r] = e4m3(k_in[i] / s), k_scale[r] = s =
+    amax / 448, kv[r] = kv_in[i], r the row of (tok_seq[i], tok_pos[i]) through the block table.
+    k_in is fp32 [n_new, idx_dim]; kv_in bf16 bits [n_new, d_kv] or None."""
+    st = lib().dsa_cache_append(ctypes.byref(cache), _ptr(k8), _ptr(k_scale), _ptr(kv),
+                                tok_seq.shape[0], _ptr(tok_seq), _ptr(tok_pos), _ptr(k_in),
+                                _ptr(kv_in), _stream(stream))
+    _check("dsa_cache_append", st)
 
 
 def dsa_read_device_status(stream=None) -> int:
