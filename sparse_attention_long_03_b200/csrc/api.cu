@@ -281,6 +281,9 @@ dsa_status dsa_forward(const dsa_paged_cache* cache, const dsa_queries* queries,
   float* logits = reinterpret_cast<float*>(ws + FL.logits);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + FL.idx);
   IndexerLaunch IL{cache, queries, q8, q_scale, w, n_idx_heads, logits, FL.ld, ws + FL.plan, st};
+  // a token with at most k valid keys selects all of them: its logits are never read, so
+  // the indexer skips it (for the first k positions a prefill is dense attention)
+  IL.skip_below = k;
   if (FL.decode) {
     // few long rows: the indexer also builds the first-digit histogram and the top-k
     // spreads each row over several CTAs

@@ -62,6 +62,9 @@ struct IndexerLaunch {
   uint32_t* hist = nullptr;     // optional [T][2048] first-digit histogram of the logits
   uint32_t* zero = nullptr;     // region the prep kernel zeroes first (histogram, counters)
   int64_t zero_words = 0;
+  // query tokens with tok_pos < skip_below get no logits (the forward selects all of their
+  // keys without reading any); 0: every token is scored
+  int32_t skip_below = 0;
 };
 cudaError_t launch_indexer(const IndexerLaunch& a);
 

@@ -100,7 +100,8 @@ __global__ void __launch_bounds__(1024) indexer_prep_kernel(const int32_t* __res
                                                             int32_t T, int32_t batch,
                                                             int32_t max_pos, int32_t pos_cap,
                                                             void* ws, uint32_t* zero,
-                                                            int64_t zero_words, int run_tokens) {
+                                                            int64_t zero_words, int run_tokens,
+                                                            int32_t skip_below) {
   __shared__ int sm[33];
   pdl_wait();
   pdl_trigger();
@@ -127,6 +128,8 @@ __global__ void __launch_bounds__(1024) indexer_prep_kernel(const int32_t* __res
           uniform = false;
         }
         if (seqs[j] != seqs[0]) uniform = false;
+        if (ok[j] && poss[j] < skip_below) ok[j] = false;  // selected whole: no logits
+
       }
       nr = uniform ? 1 : cnt;
     }
@@ -134,8 +137,9 @@ __global__ void __launch_bounds__(1024) indexer_prep_kernel(const int32_t* __res
     const int off = block_excl_scan(nr, &total, sm) + carry;
     if (g < n_groups) {
       if (uniform) {
-        int mp = poss[0];
-        for (int j = 1; j < cnt; ++j) mp = max(mp, poss[j]);
+        int mp = -1;  // no work when every token of the run is skipped
+        for (int j = 0; j < cnt; ++j)
+          if (ok[j]) mp = max(mp, poss[j]);
         v.tok0[off] = G * g;
         v.ntok[off] = cnt;
         v.seq[off] = seqs[0];
@@ -189,6 +193,7 @@ struct IdxArgs {
   void* plan;  // the prep kernel's plan, or null: the kernel plans one-token runs itself
   int32_t T;
   uint32_t* hist;  // [T][2048] first-digit histogram of the ordered logits, or null
+  int32_t skip_below;  // tokens with tok_pos below this get no logits
   int inject;      // test hook: the CTA owning item 0 skips its first stage's arrivals
 };
 
@@ -537,6 +542,8 @@ __global__ void __launch_bounds__(kIdxThreadsBound, 1)
             if (blockIdx.x == 0) record_error(kErrBadIndex);
             seq = 0;
             pos = -1;  // no work for an invalid token
+          } else if (pos < a.skip_below) {
+            pos = -1;  // selected whole: no logits
           }
           ni = (pos + kKeyTile) / kKeyTile;
         }
@@ -796,6 +803,7 @@ static cudaError_t launch_indexer_t(const IndexerLaunch& L, const CUtensorMap& m
   a.plan = RT == 1 && L.queries->n_tokens <= kInlinePlanMax ? nullptr : L.ws;
   a.T = L.queries->n_tokens;
   a.hist = L.hist;
+  a.skip_below = L.skip_below;
   a.inject = take_injection(1);
   return launch_pdl(indexer_kernel<DI, HP, RT>, dim3(grid), dim3(kIdxThreads), C::kSmemAlloc, L.stream,
                     map, a);
@@ -814,7 +822,8 @@ cudaError_t launch_indexer(const IndexerLaunch& L) {
   const bool inline_plan = RT == 1 && T <= kInlinePlanMax;
   cudaError_t e = launch_pdl(indexer_prep_kernel, dim3(1), dim3(1024), 0, L.stream, q->tok_seq,
                              q->tok_pos, T, c->batch, q->max_pos, c->max_blocks_per_seq * kPage,
-                             inline_plan ? nullptr : L.ws, L.zero, L.zero_words, RT);
+                             inline_plan ? nullptr : L.ws, L.zero, L.zero_words, RT,
+                             L.skip_below);
   if (e != cudaSuccess) return e;
 
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
