@@ -174,6 +174,44 @@ DSA_API dsa_status dsa_cache_append(const dsa_paged_cache* cache, uint8_t* k8, f
                                     const int32_t* tok_pos, const float* k_in,
                                     const uint16_t* kv_in, void* stream);
 
+/* Context-parallel decode of one long sequence (the steps between collectives).  Each of
+ * n_parts ranks owns a contiguous, page-aligned range [begin, end) of the sequence's
+ * positions, runs dsa_indexer_logits and dsa_topk over its own keys (positions local to
+ * the range), and exchanges candidates; every rank then merges them to the same global
+ * selection (section "FP8 index -> top-k selection -> sparse core attention", item (2):
+ * the k largest index scores), attends over the selected rows it owns, and the ranks'
+ * partial outputs are combined by log-sum-exp.                                           */
+
+/* Candidates of a local selection: values[t, j] = logits[t * ld + idx[t, j]] and
+ * positions[t, j] = idx[t, j] + pos_offset; an empty slot (idx < 0) gives -inf and -1.
+ * idx, values, positions device [n_tokens, k].                                            */
+DSA_API dsa_status dsa_cp_candidates(const float* logits, int64_t ld_logits, int32_t n_tokens,
+                                     const int32_t* idx, int32_t k, int32_t pos_offset,
+                                     float* values, int32_t* positions, void* stream);
+
+/* Merge: values, positions device [n_parts, n_tokens, k] (part-major, as an all-gather
+ * leaves them) -> idx_out device [n_tokens, k], the k candidates of each query with the
+ * largest values (global positions, -1 in empty slots).  Equal values go to the earlier
+ * candidate (part order, then slot order): the smaller position when each part keeps equal
+ * values in position order (dsa_topk outputs do) and parts come in the order of their
+ * ranges.  idx_local (nullable) [n_tokens, k] receives the same selection seen by the part
+ * owning [local_begin, local_end): position - local_begin there, -1 elsewhere.
+ * n_parts * k <= 32768.  Workspace: dsa_cp_merge_workspace_size bytes, 256-B aligned.    */
+DSA_API dsa_status dsa_cp_merge_topk(const float* values, const int32_t* positions,
+                                     int32_t n_parts, int32_t n_tokens, int32_t k,
+                                     int32_t* idx_out, int32_t local_begin, int32_t local_end,
+                                     int32_t* idx_local, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+DSA_API size_t dsa_cp_merge_workspace_size(int32_t n_tokens, int32_t n_parts, int32_t k);
+
+/* Combine: o_parts device bf16 [n_parts, n_tokens, n_heads, d_v], each normalised by its own
+ * softmax sum (a dsa_sparse_mla_attn output), lse_parts device fp32 [n_parts, n_tokens,
+ * n_heads] (-inf: no keys) -> out bf16 [n_tokens, n_heads, d_v] = sum_g exp(lse_g - LSE) O_g,
+ * lse (nullable) fp32 [n_tokens, n_heads] = LSE = logsumexp_g lse_g.  d_v a multiple of 4. */
+DSA_API dsa_status dsa_cp_attn_merge(const uint16_t* o_parts, const float* lse_parts,
+                                     int32_t n_parts, int32_t n_tokens, int32_t n_heads,
+                                     int32_t d_v, uint16_t* out, float* lse, void* stream);
+
 /* Waits for `stream`, then returns and clears the device status word of the current
  * device (DSA_OK, DSA_ERR_BAD_INDEX or DSA_ERR_TIMEOUT; DSA_ERR_CUDA if the wait failed). */
 DSA_API dsa_status dsa_read_device_status(void* stream);

@@ -1,0 +1,144 @@
+"""Context-parallel decode of long sequences: the keys of every sequence are split over G
+parts (ranks), each holding a contiguous, page-aligned range of positions.
+
+"DeepSeek V3.2-Exp Cuts Prolonged-Context Costs ...", section "FP8 index -> top-k
+selection -> sparse core attention": the indexer scores every preceding token, the top-k
+keeps the k best, attention runs over those.  Split over parts, one decode step is
+
+  1. on each part: dsa_indexer_logits and dsa_topk over its own keys (local positions,
+     the query's position clamped to the part's range), then dsa_cp_candidates: the
+     (logit, global position) pairs of the local selection;
+  2. exchange the candidates (all-gather, part-major);
+  3. on each part: dsa_cp_merge_topk, the same global selection everywhere plus the
+     part's local view of it, then dsa_sparse_mla_attn over the selected rows it owns:
+     a partial output normalised by its own softmax sum, and its LSE;
+  4. exchange the partials and LSEs (all-gather);
+  5. dsa_cp_attn_merge: out = sum_g exp(lse_g - LSE) O_g, LSE = logsumexp_g lse_g.
+
+The exchanges move G * T * k * 8 bytes of candidates and G * T * H * (2 d_v + 4) bytes of
+partials; every step in between runs in libdsa's kernels.  `CudaOps` binds those kernels;
+`run_parts` drives all parts of one process in order (one GPU, or a test), and
+`cp_decode_step` runs one part per rank over a torch.distributed process group.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import List, Optional
+
+import torch
+
+from . import dsa
+
+PAGE = 64
+
+
+@dataclass
+class Part:
+    """One part of the key range: positions [begin, end) of every sequence, held in a paged
+    cache whose block table maps the part's local positions 0 .. end - begin - 1."""
+    begin: int
+    end: int
+    cache: dsa.PagedCache
+
+
+@dataclass
+class Step:
+    """One decode step's query inputs (device tensors, as for dsa_forward) and sizes."""
+    tok_seq: torch.Tensor
+    tok_pos: torch.Tensor     # global positions
+    tok_pos_host: List[int]
+    q8: torch.Tensor
+    q_scale: torch.Tensor
+    w: torch.Tensor
+    q: torch.Tensor
+    n_heads: int
+    d_v: int
+    scale: float
+    k: int
+
+
+class CudaOps:
+    """The step's kernels, through the libdsa binding."""
+
+    def local_candidates(self, part: Part, st: Step):
+        T = st.tok_seq.shape[0]
+        dev = st.q8.device
+        local_pos = [min(p, part.end - 1) - part.begin for p in st.tok_pos_host]
+        if min(local_pos) < 0:
+            raise ValueError("every query needs at least one key in every part")
+        tok_pos = torch.tensor(local_pos, dtype=torch.int32, device=dev)
+        queries = dsa.make_queries(st.tok_seq, tok_pos, max(local_pos))
+        ld = ((max(local_pos) + 1 + 127) // 128) * 128
+        logits = torch.empty((T, ld), dtype=torch.float32, device=dev)
+        dsa.dsa_indexer_logits(part.cache, queries, st.q8, st.q_scale, st.w, logits)
+        idx = torch.empty((T, st.k), dtype=torch.int32, device=dev)
+        dsa.dsa_topk(logits, queries, st.k, idx)
+        values = torch.empty((T, st.k), dtype=torch.float32, device=dev)
+        positions = torch.empty((T, st.k), dtype=torch.int32, device=dev)
+        dsa.dsa_cp_candidates(logits, idx, part.begin, values, positions)
+        return values, positions, queries
+
+    def merge_and_attend(self, part: Part, st: Step, values, positions, queries):
+        T = st.tok_seq.shape[0]
+        dev = st.q8.device
+        idx = torch.empty((T, st.k), dtype=torch.int32, device=dev)
+        idx_local = torch.empty((T, st.k), dtype=torch.int32, device=dev)
+        dsa.dsa_cp_merge_topk(values, positions, st.k, idx, part.begin, part.end, idx_local)
+        out = torch.empty((T, st.n_heads, st.d_v), dtype=torch.int16, device=dev)
+        lse = torch.empty((T, st.n_heads), dtype=torch.float32, device=dev)
+        dsa.dsa_sparse_mla_attn(part.cache, queries, st.q, st.d_v, st.scale, idx_local, out, lse)
+        return idx, out, lse
+
+    def combine(self, o_parts, lse_parts):
+        G, T, H, d_v = o_parts.shape
+        out = torch.empty((T, H, d_v), dtype=torch.int16, device=o_parts.device)
+        lse = torch.empty((T, H), dtype=torch.float32, device=o_parts.device)
+        dsa.dsa_cp_attn_merge(o_parts, lse_parts, out, lse)
+        return out, lse
+
+
+def run_parts(parts: List[Part], st: Step, ops: Optional[CudaOps] = None):
+    """All parts in one process, in order (the exchanges are stacks).  Returns the global
+    selection (logical positions), out and LSE."""
+    ops = ops or CudaOps()
+    local = [ops.local_candidates(p, st) for p in parts]
+    values = torch.stack([v for v, _, _ in local])
+    positions = torch.stack([x for _, x, _ in local])
+    res = [ops.merge_and_attend(p, st, values, positions, lq) for p, (_, _, lq) in zip(parts, local)]
+    out, lse = ops.combine(torch.stack([o for _, o, _ in res]), torch.stack([l for _, _, l in res]))
+    return res[0][0], out, lse
+
+
+def cp_decode_step(part: Part, st: Step, group=None, ops: Optional[CudaOps] = None):
+    """This rank's part of one decode step over a torch.distributed group (parts in rank
+    order).  Every rank returns the same selection, out and LSE."""
+    import torch.distributed as dist
+    ops = ops or CudaOps()
+    G = dist.get_world_size(group)
+
+    def gather(x):  # part-major stack of every rank's tensor (gloo and nccl both take lists)
+        xs = [torch.empty_like(x) for _ in range(G)]
+        dist.all_gather(xs, x.contiguous(), group=group)
+        return torch.stack(xs)
+
+    values, positions, queries = ops.local_candidates(part, st)
+    all_v, all_p = gather(values), gather(positions)
+    idx, o, l = ops.merge_and_attend(part, st, all_v, all_p, queries)
+    all_o, all_l = gather(o), gather(l)
+    out, lse = ops.combine(all_o, all_l)
+    return idx, out, lse
+
+
+def split_parts(block_table: torch.Tensor, k8, k_scale, kv, lengths: List[int], G: int):
+    """Parts of a shared physical cache: part g owns the page-aligned position range
+    [g * P, (g + 1) * P) of every sequence (P = the longest length split G ways, rounded up
+    to whole pages); its block table is the matching column slice of `block_table`."""
+    n_pages = (max(lengths) + PAGE - 1) // PAGE
+    per = (n_pages + G - 1) // G
+    parts = []
+    for g in range(G):
+        c0, c1 = g * per, min((g + 1) * per, block_table.shape[1])
+        bt = block_table[:, c0:c1].contiguous()
+        parts.append(Part(c0 * PAGE, c1 * PAGE, dsa.make_cache(k8, k_scale, kv, bt)))
+    return parts

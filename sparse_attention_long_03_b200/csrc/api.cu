@@ -167,6 +167,50 @@ dsa_status dsa_cache_append(const dsa_paged_cache* cache, uint8_t* k8, float* k_
                                          static_cast<cudaStream_t>(stream)));
 }
 
+dsa_status dsa_cp_candidates(const float* logits, int64_t ld_logits, int32_t n_tokens,
+                             const int32_t* idx, int32_t k, int32_t pos_offset, float* values,
+                             int32_t* positions, void* stream) {
+  using namespace dsa;
+  if (n_tokens < 0 || k < 1 || k > kMaxTopK || ld_logits < 1) return DSA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return DSA_OK;
+  if (!logits || !idx || !values || !positions) return DSA_ERR_INVALID_ARG;
+  return cuda_status(launch_cp_candidates(logits, ld_logits, n_tokens, idx, k, pos_offset,
+                                          values, positions, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dsa_cp_merge_workspace_size(int32_t n_tokens, int32_t n_parts, int32_t k) {
+  if (n_tokens <= 0 || n_parts <= 0 || k <= 0) return 0;
+  return dsa::cp_merge_ws_bytes(n_tokens, n_parts, k);
+}
+
+dsa_status dsa_cp_merge_topk(const float* values, const int32_t* positions, int32_t n_parts,
+                             int32_t n_tokens, int32_t k, int32_t* idx_out, int32_t local_begin,
+                             int32_t local_end, int32_t* idx_local, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  using namespace dsa;
+  if (n_tokens < 0 || n_parts < 1 || k < 1 || k > kMaxTopK) return DSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(n_parts) * k > 32768) return DSA_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return DSA_OK;
+  if (!values || !positions || !idx_out || !workspace) return DSA_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return DSA_ERR_INVALID_ARG;
+  if (workspace_bytes < cp_merge_ws_bytes(n_tokens, n_parts, k)) return DSA_ERR_WORKSPACE;
+  return cuda_status(launch_cp_merge(values, positions, n_parts, n_tokens, k, idx_out,
+                                     local_begin, local_end, idx_local, workspace,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_cp_attn_merge(const uint16_t* o_parts, const float* lse_parts, int32_t n_parts,
+                             int32_t n_tokens, int32_t n_heads, int32_t d_v, uint16_t* out,
+                             float* lse, void* stream) {
+  using namespace dsa;
+  if (n_parts < 1 || n_tokens < 0 || n_heads < 1 || d_v < 4 || d_v % 4) return DSA_ERR_INVALID_ARG;
+  if (n_tokens == 0) return DSA_OK;
+  if (!o_parts || !lse_parts || !out) return DSA_ERR_INVALID_ARG;
+  if (!aligned(o_parts, 8) || !aligned(out, 8)) return DSA_ERR_INVALID_ARG;
+  return cuda_status(launch_cp_attn_merge(o_parts, lse_parts, n_parts, n_tokens, n_heads, d_v,
+                                          out, lse, static_cast<cudaStream_t>(stream)));
+}
+
 int32_t dsa_last_cuda_error(void) { return g_last_cuda_error.load(); }
 
 dsa_status dsa_debug_inject(int32_t fault) {

@@ -1,0 +1,192 @@
+// Context-parallel decode of one long sequence: the steps between the ranks' collectives.
+//
+// Each of G ranks owns a contiguous, page-aligned range [begin, end) of a sequence's
+// positions and runs the indexer and a local top-k over its own keys.  The k best local
+// entries are exchanged as (logit, position) candidates; every rank merges the G * k
+// candidates of a query to the same global top-k ("DeepSeek V3.2-Exp Cuts Prolonged-Context
+// Costs ...", section "FP8 index -> top-k selection -> sparse core attention", item (2):
+// the k entries with the largest index scores), attends over the selected rows it owns,
+// and the G normalised partial outputs are combined by their log-sum-exp.
+//
+//   candidates  idx (local positions) -> logits at them and global positions
+//   merge       [G, T, k] candidates -> [T, k] global selection (+ this rank's local view)
+//   attn merge  [G, T, H, d_v] bf16 partials + [G, T, H] LSE -> out, LSE
+//
+// The merge reuses the per-row top-k on each query's G * k candidate values; equal values
+// go to the earlier candidate slot, which is the smaller position when each rank's list
+// keeps equal values in position order (a dsa_topk output does) and ranks come in the order
+// of their ranges.
+#include <cuda_fp16.h>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+__global__ void __launch_bounds__(256) cp_candidates_kernel(const float* __restrict__ logits,
+                                                            int64_t ld,
+                                                            const int32_t* __restrict__ idx,
+                                                            int64_t n, int32_t k, int32_t offset,
+                                                            float* __restrict__ values,
+                                                            int32_t* __restrict__ positions) {
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = e / k;
+    const int p = idx[e];
+    values[e] = p >= 0 ? logits[t * ld + p] : -INFINITY;
+    positions[e] = p >= 0 ? p + offset : -1;
+  }
+}
+
+// [G, T, k] -> one row of G * k candidates per query; every row has G * k valid entries
+__global__ void __launch_bounds__(256) cp_merge_rows_kernel(
+    const float* __restrict__ values, const int32_t* __restrict__ positions, int32_t G,
+    int32_t T, int32_t k, float* __restrict__ vrows, int32_t* __restrict__ prows,
+    int32_t* __restrict__ row_pos, int32_t* __restrict__ row_seq) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t nc = static_cast<int64_t>(G) * k;
+  const int64_t n = static_cast<int64_t>(T) * nc;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = e / nc, rem = e % nc, g = rem / k, j = rem % k;
+    const int64_t src = (g * T + t) * k + j;
+    vrows[e] = values[src];
+    prows[e] = positions[src];
+    if (rem == 0) {
+      row_pos[t] = static_cast<int32_t>(nc - 1);
+      row_seq[t] = 0;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) cp_merge_map_kernel(
+    const int32_t* __restrict__ slots, const int32_t* __restrict__ prows, int32_t T,
+    int64_t nc, int32_t k, int32_t* __restrict__ idx_out, int32_t local_begin,
+    int32_t local_end, int32_t* __restrict__ idx_local) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t n = static_cast<int64_t>(T) * k;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = e / k;
+    const int s = slots[e];
+    const int p = s >= 0 ? prows[t * nc + s] : -1;
+    idx_out[e] = p;
+    if (idx_local) idx_local[e] = (p >= local_begin && p < local_end) ? p - local_begin : -1;
+  }
+}
+
+// O = sum_g exp(lse_g - LSE) O_g, LSE = logsumexp_g lse_g; one CTA per (head, token), four
+// dims per thread, every part's loads issued together, folded under a running maximum.
+__global__ void __launch_bounds__(128) cp_attn_merge_kernel(
+    const uint16_t* __restrict__ o_parts, const float* __restrict__ lse_parts, int32_t G,
+    int32_t T, int32_t H, int32_t d_v, uint16_t* __restrict__ out, float* __restrict__ lse) {
+  pdl_wait();
+  pdl_trigger();
+  const int t = blockIdx.y, h = blockIdx.x;
+  const size_t part = static_cast<size_t>(T) * H;  // (t, h) rows per part
+  for (int d = threadIdx.x * 4; d < d_v; d += blockDim.x * 4) {
+    float m = -INFINITY, sum = 0.f;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    constexpr int kBatch = 8;
+    for (int g0 = 0; g0 < G; g0 += kBatch) {
+      float ls[kBatch];
+      uint2 v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const bool in = g0 + u < G;
+        const size_t row = (g0 + u) * part + static_cast<size_t>(t) * H + h;
+        ls[u] = in ? lse_parts[row] : -INFINITY;
+        v[u] = in ? *reinterpret_cast<const uint2*>(o_parts + row * d_v + d) : make_uint2(0, 0);
+      }
+      float mb = m;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) mb = fmaxf(mb, ls[u]);
+      if (mb == -INFINITY) continue;
+      const float sc = m == -INFINITY ? 0.f : __expf(m - mb);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[c] *= sc;
+      sum *= sc;
+      m = mb;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const float e = ls[u] == -INFINITY ? 0.f : __expf(ls[u] - m);
+        sum += e;
+        const uint32_t w0 = v[u].x, w1 = v[u].y;  // four bf16
+        acc[0] = fmaf(e, __uint_as_float(w0 << 16), acc[0]);
+        acc[1] = fmaf(e, __uint_as_float(w0 & 0xFFFF0000u), acc[1]);
+        acc[2] = fmaf(e, __uint_as_float(w1 << 16), acc[2]);
+        acc[3] = fmaf(e, __uint_as_float(w1 & 0xFFFF0000u), acc[3]);
+      }
+    }
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
+    *reinterpret_cast<uint2*>(out + (static_cast<size_t>(t) * H + h) * d_v + d) =
+        make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+    if (d == 0 && lse) lse[static_cast<size_t>(t) * H + h] = sum > 0.f ? m + __logf(sum) : -INFINITY;
+  }
+}
+
+int grid_for(int64_t n) {
+  const int64_t g = (n + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  return static_cast<int>(g < 1 ? 1 : (g < cap ? g : cap));
+}
+
+size_t al(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+size_t cp_merge_ws_bytes(int32_t T, int32_t G, int32_t k) {
+  const size_t nc = static_cast<size_t>(G) * k;
+  return al(static_cast<size_t>(T) * nc * 4) * 2 + al(static_cast<size_t>(T) * 4) * 2 +
+         al(static_cast<size_t>(T) * k * 4);
+}
+
+cudaError_t launch_cp_candidates(const float* logits, int64_t ld, int32_t T, const int32_t* idx,
+                                 int32_t k, int32_t offset, float* values, int32_t* positions,
+                                 cudaStream_t stream) {
+  const int64_t n = static_cast<int64_t>(T) * k;
+  if (n == 0) return cudaSuccess;
+  return launch_pdl(cp_candidates_kernel, dim3(grid_for(n)), dim3(256), 0, stream, logits, ld,
+                    idx, n, k, offset, values, positions);
+}
+
+cudaError_t launch_cp_merge(const float* values, const int32_t* positions, int32_t G, int32_t T,
+                            int32_t k, int32_t* idx_out, int32_t local_begin, int32_t local_end,
+                            int32_t* idx_local, void* ws, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const int64_t nc = static_cast<int64_t>(G) * k;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  float* vrows = reinterpret_cast<float*>(p);
+  p += al(static_cast<size_t>(T) * nc * 4);
+  int32_t* prows = reinterpret_cast<int32_t*>(p);
+  p += al(static_cast<size_t>(T) * nc * 4);
+  int32_t* row_pos = reinterpret_cast<int32_t*>(p);
+  p += al(static_cast<size_t>(T) * 4);
+  int32_t* row_seq = reinterpret_cast<int32_t*>(p);
+  p += al(static_cast<size_t>(T) * 4);
+  int32_t* slots = reinterpret_cast<int32_t*>(p);
+  cudaError_t e = launch_pdl(cp_merge_rows_kernel, dim3(grid_for(T * nc)), dim3(256), 0, stream,
+                             values, positions, G, T, k, vrows, prows, row_pos, row_seq);
+  if (e != cudaSuccess) return e;
+  // the k best of each row of candidates (rows are all valid: positions 0..G*k-1)
+  dsa_queries rows{T, row_seq, row_pos, static_cast<int32_t>(nc - 1)};
+  e = launch_topk(vrows, nc, &rows, k, slots, nullptr, stream);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(cp_merge_map_kernel, dim3(grid_for(static_cast<int64_t>(T) * k)), dim3(256), 0,
+                    stream, slots, prows, T, nc, k, idx_out, local_begin, local_end, idx_local);
+}
+
+cudaError_t launch_cp_attn_merge(const uint16_t* o_parts, const float* lse_parts, int32_t G,
+                                 int32_t T, int32_t H, int32_t d_v, uint16_t* out, float* lse,
+                                 cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  return launch_pdl(cp_attn_merge_kernel, dim3(H, T), dim3(128), 0, stream, o_parts, lse_parts,
+                    G, T, H, d_v, out, lse);
+}
+
+}  // namespace dsa

@@ -40,6 +40,18 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return e;
 }
 
+// ---- context-parallel decode ----------------------------------------------------------
+size_t cp_merge_ws_bytes(int32_t T, int32_t G, int32_t k);
+cudaError_t launch_cp_candidates(const float* logits, int64_t ld, int32_t T, const int32_t* idx,
+                                 int32_t k, int32_t offset, float* values, int32_t* positions,
+                                 cudaStream_t stream);
+cudaError_t launch_cp_merge(const float* values, const int32_t* positions, int32_t G, int32_t T,
+                            int32_t k, int32_t* idx_out, int32_t local_begin, int32_t local_end,
+                            int32_t* idx_local, void* ws, cudaStream_t stream);
+cudaError_t launch_cp_attn_merge(const uint16_t* o_parts, const float* lse_parts, int32_t G,
+                                 int32_t T, int32_t H, int32_t d_v, uint16_t* out, float* lse,
+                                 cudaStream_t stream);
+
 // ---- cache append -------------------------------------------------------------------
 cudaError_t launch_cache_append(const dsa_paged_cache* c, uint8_t* k8, float* k_scale,
                                 uint16_t* kv, int32_t n_new, const int32_t* tok_seq,

@@ -509,10 +509,35 @@ __global__ void __launch_bounds__(kTopkDecThreads, 1)
     for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
     return;
   }
-  // the finals, in chunk order: all loads first, then the stores
+  // The finals (in chunk order) and the first batch of candidates: every load is issued
+  // before any store, so the two gathers share one round trip.
   constexpr int kFin = (kMaxTopK + kTopkDecThreads - 1) / kTopkDecThreads;
+  constexpr int kCandBatch = 4;
+  const bool cand_in_smem = got_b <= kTopkCand;
+  auto load_cands = [&](int g0, int2* cv) {
+#pragma unroll
+    for (int u = 0; u < kCandBatch; ++u) {
+      const int g = g0 + u * kTopkDecThreads + threadIdx.x;
+      cv[u] = make_int2(0, 0);
+      if (g < got_b) {
+        const int cc = chunk_of(sm->pre_b, g);
+        cv[u] = sb[chunk_start(cc) + g - sm->pre_b[cc]];
+      }
+    }
+  };
+  auto store_cands = [&](int g0, const int2* cv) {
+#pragma unroll
+    for (int u = 0; u < kCandBatch; ++u) {
+      const int g = g0 + u * kTopkDecThreads + threadIdx.x;
+      if (g < got_b) {
+        sm->cand_idx[g] = cv[u].x;
+        sm->cand_key[g] = static_cast<uint32_t>(cv[u].y);
+      }
+    }
+  };
   {
     int32_t v[kFin];
+    int2 cv[kCandBatch];
 #pragma unroll
     for (int u = 0; u < kFin; ++u) {
       const int g = u * kTopkDecThreads + threadIdx.x;
@@ -522,32 +547,19 @@ __global__ void __launch_bounds__(kTopkDecThreads, 1)
         v[u] = sa[chunk_start(cc) + g - sm->pre_a[cc]];
       }
     }
+    if (cand_in_smem) load_cands(0, cv);
 #pragma unroll
     for (int u = 0; u < kFin; ++u) {
       const int g = u * kTopkDecThreads + threadIdx.x;
       if (g < got_a) out[g] = v[u];
     }
+    if (cand_in_smem) store_cands(0, cv);
   }
-  if (got_b <= kTopkCand) {
-    for (int g0 = 0; g0 < got_b; g0 += 4 * kTopkDecThreads) {
-      int2 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int g = g0 + u * kTopkDecThreads + threadIdx.x;
-        v[u] = make_int2(0, 0);
-        if (g < got_b) {
-          const int cc = chunk_of(sm->pre_b, g);
-          v[u] = sb[chunk_start(cc) + g - sm->pre_b[cc]];
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int g = g0 + u * kTopkDecThreads + threadIdx.x;
-        if (g < got_b) {
-          sm->cand_idx[g] = v[u].x;
-          sm->cand_key[g] = static_cast<uint32_t>(v[u].y);
-        }
-      }
+  if (cand_in_smem) {
+    for (int g0 = kCandBatch * kTopkDecThreads; g0 < got_b; g0 += kCandBatch * kTopkDecThreads) {
+      int2 cv[kCandBatch];
+      load_cands(g0, cv);
+      store_cands(g0, cv);
     }
     __syncthreads();
     finish_candidates(sm, RowCand{sm->cand_key, sm->cand_idx}, got_b, b1, k2, out + got_a);

@@ -29,7 +29,9 @@ EXPORTED = ("dsa_indexer_logits", "dsa_indexer_workspace_size", "dsa_indexer_log
             "dsa_topk_workspace_size", "dsa_sparse_mla_attn", "dsa_attn_workspace_size",
             "dsa_forward", "dsa_forward_workspace_size", "dsa_read_device_status",
             "dsa_launch_count", "dsa_status_string", "dsa_abi_version", "dsa_debug_inject",
-            "dsa_debug_timeout_site", "dsa_last_cuda_error", "dsa_cache_append")
+            "dsa_debug_timeout_site", "dsa_last_cuda_error", "dsa_cache_append",
+            "dsa_cp_candidates", "dsa_cp_merge_topk", "dsa_cp_merge_workspace_size",
+            "dsa_cp_attn_merge")
 
 
 class DsaError(RuntimeError):
@@ -94,6 +96,10 @@ def lib() -> ctypes.CDLL:
             "dsa_debug_timeout_site": (ctypes.c_uint32, []),
             "dsa_last_cuda_error": (I32, []),
             "dsa_cache_append": (I32, [PC, P, P, P, I32, P, P, P, P, P]),
+            "dsa_cp_candidates": (I32, [P, I64, I32, P, I32, I32, P, P, P]),
+            "dsa_cp_merge_topk": (I32, [P, P, I32, I32, I32, P, I32, I32, P, P, SZ, P]),
+            "dsa_cp_merge_workspace_size": (SZ, [I32, I32, I32]),
+            "dsa_cp_attn_merge": (I32, [P, P, I32, I32, I32, I32, P, P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -232,6 +238,39 @@ def dsa_cache_append(cache: PagedCache, k8, k_scale, kv, tok_seq, tok_pos, k_in,
                                 tok_seq.shape[0], _ptr(tok_seq), _ptr(tok_pos), _ptr(k_in),
                                 _ptr(kv_in), _stream(stream))
     _check("dsa_cache_append", st)
+
+
+def dsa_cp_candidates(logits, idx, pos_offset: int, values, positions, stream=None):
+    """values[t, j] = logits[t, idx[t, j]], positions[t, j] = idx[t, j] + pos_offset (-inf / -1
+    for empty slots)."""
+    T, k = idx.shape
+    _check("dsa_cp_candidates",
+           lib().dsa_cp_candidates(_ptr(logits), logits.shape[1], T, _ptr(idx), k,
+                                   int(pos_offset), _ptr(values), _ptr(positions),
+                                   _stream(stream)))
+
+
+def dsa_cp_merge_topk(values, positions, k: int, idx_out, local_begin: int = 0,
+                      local_end: int = 0, idx_local=None, workspace=None, stream=None):
+    """[G, T, k] candidates -> [T, k] global selection (and this part's local view)."""
+    G, T, kc = values.shape
+    need = int(lib().dsa_cp_merge_workspace_size(T, G, kc))
+    if workspace is None:
+        workspace = _workspace(need, values.device)
+    _check("dsa_cp_merge_topk",
+           lib().dsa_cp_merge_topk(_ptr(values), _ptr(positions), G, T, k, _ptr(idx_out),
+                                   int(local_begin), int(local_end), _ptr(idx_local),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)))
+    return idx_out
+
+
+def dsa_cp_attn_merge(o_parts, lse_parts, out, lse=None, stream=None):
+    """[G, T, H, d_v] bf16 partials + [G, T, H] LSE -> out [T, H, d_v], lse [T, H]."""
+    G, T, H, d_v = o_parts.shape
+    _check("dsa_cp_attn_merge",
+           lib().dsa_cp_attn_merge(_ptr(o_parts), _ptr(lse_parts), G, T, H, d_v, _ptr(out),
+                                   _ptr(lse), _stream(stream)))
+    return out
 
 
 def dsa_read_device_status(stream=None) -> int:

@@ -1,0 +1,132 @@
+"""Context-parallel decode plumbing on CPU: two gloo ranks, each owning half of every
+sequence's positions, run cp_decode_step with the float64 oracle standing in for the
+kernels.  The merged selection must equal the oracle's single-part top-k exactly and the
+log-sum-exp merge of the two partial attentions must equal its attention over the whole
+selection: local top-k + exchange + merge is the global top-k, and the partial outputs
+recombine without loss."""
+
+import os
+import socket
+
+import numpy as np
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+class OraclePart:
+    def __init__(self, begin, end, bt):
+        self.begin, self.end, self.bt = begin, end, bt
+
+
+class OracleOps:
+    """float64 stand-ins for the kernels of one part (CPU tensors in, CPU tensors out)."""
+
+    def __init__(self, cfg, cache, qs):
+        self.cfg, self.cache, self.qs = cfg, cache, qs
+
+    def local_candidates(self, part, st):
+        from oracle import dsa_ref as R
+        T, k = len(st.tok_pos_host), st.k
+        vals = np.full((T, k), -np.inf)
+        poss = np.full((T, k), -1, np.int32)
+        local = [min(p, part.end - 1) - part.begin for p in st.tok_pos_host]
+        for t in range(T):
+            b = int(self.qs.tok_seq[t])
+            row = R.indexer_logits_row(self.cache.k8, self.cache.k_scale, part.bt, b, local[t],
+                                       self.qs.q8[t], self.qs.q_scale[t], self.qs.w[t])
+            sel = R.topk_select(row, k)
+            vals[t, :len(sel)] = row[sel]
+            poss[t, :len(sel)] = sel + part.begin
+        return torch.from_numpy(vals), torch.from_numpy(poss), local
+
+    def merge_and_attend(self, part, st, values, positions, local):
+        from oracle import dsa_ref as R
+        G, T, k = values.shape
+        H, dv = self.cfg.n_heads, self.cfg.d_v
+        idx = np.full((T, k), -1, np.int32)
+        O = np.zeros((T, H, dv))
+        L = np.full((T, H), -np.inf)
+        for t in range(T):
+            v = values[:, t, :].reshape(-1).numpy()
+            p = positions[:, t, :].reshape(-1).numpy()
+            keep = p >= 0
+            v, p = v[keep], p[keep]
+            order = np.lexsort((p, -v))[:k]  # larger value first, then the smaller position
+            sel = np.sort(p[order])
+            idx[t, :len(sel)] = sel
+            mine = sel[(sel >= part.begin) & (sel < part.end)] - part.begin
+            if len(mine):
+                O[t], L[t] = R.sparse_mla_attn_token(self.cache.kv, part.bt,
+                                                     int(self.qs.tok_seq[t]), self.qs.q[t], mine,
+                                                     self.cfg.scale, dv)
+        return torch.from_numpy(idx), torch.from_numpy(O), torch.from_numpy(L)
+
+    def combine(self, o_parts, lse_parts):
+        o, l = o_parts.numpy(), lse_parts.numpy()
+        m = l.max(axis=0)
+        wts = np.where(np.isfinite(l), np.exp(l - m), 0.0)
+        s = wts.sum(axis=0)
+        out = (wts[..., None] * o).sum(axis=0) / s[..., None]
+        return torch.from_numpy(out), torch.from_numpy(m + np.log(s))
+
+
+def _rank_main(rank, world, port, q):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    from oracle import dsa_ref as R
+    from sparse_attention_long_03_b200 import context_parallel as CP
+    from sparse_attention_long_03_b200 import workloads as W
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        cfg, cache, qs = W.make("tiny")
+        pages = cache.block_table.shape[1]
+        per = pages // world
+        part = OraclePart(rank * per * 64, (rank + 1) * per * 64,
+                          np.ascontiguousarray(cache.block_table[:, rank * per:(rank + 1) * per]))
+        st = CP.Step(tok_seq=None, tok_pos=None, tok_pos_host=[int(p) for p in qs.tok_pos],
+                     q8=None, q_scale=None, w=None, q=None, n_heads=cfg.n_heads, d_v=cfg.d_v,
+                     scale=cfg.scale, k=cfg.topk)
+        idx, out, lse = CP.cp_decode_step(part, st, ops=OracleOps(cfg, cache, qs))
+        errs = []
+        for t in range(qs.n_tokens):
+            b, pos = int(qs.tok_seq[t]), int(qs.tok_pos[t])
+            row = R.indexer_logits_row(cache.k8, cache.k_scale, cache.block_table, b, pos,
+                                       qs.q8[t], qs.q_scale[t], qs.w[t])
+            sel = R.topk_select(row, cfg.topk)
+            o_ref, l_ref = R.sparse_mla_attn_token(cache.kv, cache.block_table, b, qs.q[t], sel,
+                                                   cfg.scale, cfg.d_v)
+            got = idx[t].numpy()
+            errs.append((set(got[got >= 0].tolist()) == set(sel.tolist()),
+                         float(np.abs(out[t].numpy() - o_ref).max()),
+                         float(np.abs(lse[t].numpy() - l_ref).max())))
+        q.put((rank, errs))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_match_the_single_part_oracle():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+        assert p.exitcode == 0
+    got = dict(q.get(timeout=5) for _ in range(2))
+    for rank in (0, 1):
+        for same_sel, o_err, l_err in got[rank]:
+            assert same_sel
+            assert o_err < 1e-10 and l_err < 1e-10

@@ -1,0 +1,42 @@
+"""Context-parallel decode kernels on one GPU: decode 32K split into two parts (halves of
+every sequence's positions) run one after the other through run_parts.  The merged
+selection equals the single-part dsa_forward selection exactly (the parts' indexers score
+each key exactly as the whole does), and the log-sum-exp merge of the parts' partial
+outputs meets the attention tolerances against the float64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dsa_ref as R
+from sparse_attention_long_03_b200 import context_parallel as CP
+from sparse_attention_long_03_b200 import dsa
+from sparse_attention_long_03_b200 import workloads as W
+
+from dsa_testutil import (ATTN_MAX_ABS, ATTN_MEAN_REL, LSE_ABS, DeviceWorkload, attn_errors,
+                          bf16_to_f64, oracle_attention)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("G", [2, 3])
+def test_parts_match_forward_and_oracle(G):
+    cfg, cache, qs = W.make("decode_32k")
+    w = DeviceWorkload(cfg, cache, qs)
+    out_f, lse_f, idx_f = w.forward()
+    lengths = [int(p) + 1 for p in qs.tok_pos]
+    parts = CP.split_parts(w.block_table, w.k8, w.k_scale, w.kv, lengths, G)
+    st = CP.Step(tok_seq=w.tok_seq, tok_pos=w.tok_pos, tok_pos_host=[int(p) for p in qs.tok_pos],
+                 q8=w.q8, q_scale=w.q_scale, w=w.w, q=w.q, n_heads=cfg.n_heads, d_v=cfg.d_v,
+                 scale=cfg.scale, k=cfg.topk)
+    idx, out, lse = CP.run_parts(parts, st)
+    assert dsa.dsa_read_device_status() == 0
+    gi, fi = idx.cpu().numpy(), idx_f.cpu().numpy()
+    for t in range(qs.n_tokens):
+        assert set(gi[t][gi[t] >= 0].tolist()) == set(fi[t][fi[t] >= 0].tolist())
+    for t in (0, qs.n_tokens - 1):
+        sel = gi[t][gi[t] >= 0]
+        o_ref, l_ref = oracle_attention(w, t, sel)
+        mx, mr = attn_errors(bf16_to_f64(out[t]), o_ref)
+        assert mx <= ATTN_MAX_ABS and mr <= ATTN_MEAN_REL, (mx, mr)
+        assert np.abs(lse[t].cpu().numpy() - l_ref).max() <= LSE_ABS
