@@ -98,3 +98,43 @@ def test_forward_workspace_size_grows_with_context():
     b = dsa.forward_workspace_size(4, 131071, 2048, 128, 512)
     assert b > a > 4 * 65536 * 4
     assert dsa.forward_workspace_size(0, 0, 2048, 128, 512) >= 0
+
+
+def test_cache_append_validation():
+    L = dsa.lib()
+    c = _cache()
+
+    def call(cache=c, k8=16, ks=16, kv=16, n=4, seq=16, pos=16, k_in=16, kv_in=16):
+        return L.dsa_cache_append(ctypes.byref(cache) if cache is not None else None, k8, ks, kv,
+                                  n, seq, pos, k_in, kv_in, None)
+
+    assert call(cache=None) == 1
+    assert call(n=-1) == 1
+    assert call(cache=_cache(page_size=32)) == 2
+    assert call(cache=_cache(idx_dim=130)) == 1  # not a multiple of 4
+    assert call(cache=_cache(idx_dim=2048)) == 1
+    assert call(k8=None) == 1
+    assert call(k_in=None) == 1
+    assert call(k_in=24) == 1  # keys are read 16 bytes at a time
+    assert call(cache=_cache(d_kv=84)) == 1  # rows are copied 16 bytes at a time
+    assert call(n=0) == 0  # nothing to do, nothing launched
+
+
+def test_context_parallel_validation():
+    L = dsa.lib()
+    # candidates
+    assert L.dsa_cp_candidates(16, 512, 4, 16, 0, 0, 16, 16, None) == 1
+    assert L.dsa_cp_candidates(None, 512, 4, 16, 2048, 0, 16, 16, None) == 1
+    assert L.dsa_cp_candidates(16, 512, 0, 16, 2048, 0, 16, 16, None) == 0
+    # merge
+    ws = dsa.lib().dsa_cp_merge_workspace_size(4, 2, 2048)
+    assert ws >= 4 * 2 * 2048 * 8
+    assert L.dsa_cp_merge_topk(16, 16, 0, 4, 2048, 16, 0, 0, None, 256, ws, None) == 1
+    assert L.dsa_cp_merge_topk(16, 16, 32, 4, 2048, 16, 0, 0, None, 256, ws, None) == 2  # > 32768
+    assert L.dsa_cp_merge_topk(16, 16, 2, 4, 2048, 16, 0, 0, None, 256, 8, None) == 3
+    assert L.dsa_cp_merge_topk(16, 16, 2, 4, 2048, 16, 0, 0, None, 272, ws, None) == 1  # alignment
+    assert L.dsa_cp_merge_topk(16, 16, 2, 0, 2048, 16, 0, 0, None, None, 0, None) == 0
+    # attention merge
+    assert L.dsa_cp_attn_merge(16, 16, 2, 4, 128, 510, 16, None, None) == 1  # d_v % 4
+    assert L.dsa_cp_attn_merge(None, 16, 2, 4, 128, 512, 16, None, None) == 1
+    assert L.dsa_cp_attn_merge(16, 16, 2, 0, 128, 512, 16, None, None) == 0
