@@ -110,6 +110,13 @@ def lib() -> ctypes.CDLL:
 
 # ------------------------------------------------------------------------------ helpers
 
+# element types the entry points read; FP8 and BF16 data travel as raw bytes or 16-bit words
+DT_FP8 = (torch.uint8, torch.float8_e4m3fn)
+DT_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+DT_F32 = (torch.float32,)
+DT_I32 = (torch.int32,)
+
+
 def _ptr(t: Optional[torch.Tensor]):
     if t is None:
         return None
@@ -118,6 +125,33 @@ def _ptr(t: Optional[torch.Tensor]):
     if not t.is_contiguous():
         raise ValueError("libdsa takes contiguous tensors only")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _check_arg(t: Optional[torch.Tensor], name: str, dtypes, shape, optional: bool = False):
+    """What the C entry points cannot see behind a raw pointer: the element type and the
+    extents (None in ``shape``: any extent).  A tensor smaller than the call implies would
+    let a kernel read or write past its end, so a mismatch raises before any launch."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected one of {[str(d) for d in dtypes]}")
+    ts = t.shape
+    ok = len(ts) == len(shape)
+    if ok:
+        for e, n in zip(shape, ts):
+            if e is not None and e != n:
+                ok = False
+                break
+    if not ok:
+        want = tuple("*" if e is None else int(e) for e in shape)
+        raise ValueError(f"{name}: shape {tuple(ts)}, expected {want}")
+
+
+def _check_ld(t: torch.Tensor, name: str, queries: "Queries"):
+    if t.shape[1] < queries.max_pos + 1:
+        raise ValueError(f"{name}: {t.shape[1]} columns < max_pos + 1 = {queries.max_pos + 1}")
 
 
 def _stream(stream=None):
@@ -135,6 +169,11 @@ def make_cache(k8: torch.Tensor, k_scale: torch.Tensor, kv: Optional[torch.Tenso
     """Describe device caches: k8 uint8 [rows, D_I], k_scale fp32 [rows],
     kv uint16/int16/bf16 [rows, D_kv], block_table int32 [B, max_blocks]."""
     rows = k8.shape[0] if k8 is not None else kv.shape[0]
+    if k8 is not None:
+        _check_arg(k8, "k8", DT_FP8, (rows, None))
+        _check_arg(k_scale, "k_scale", DT_F32, (rows,))
+    _check_arg(kv, "kv", DT_BF16, (rows, None), optional=k8 is not None)
+    _check_arg(block_table, "block_table", DT_I32, (None, None))
     c = PagedCache(
         _ptr(k8), _ptr(k_scale), _ptr(kv), _ptr(block_table), block_table.shape[0],
         block_table.shape[1], rows // page_size, page_size,
@@ -144,9 +183,31 @@ def make_cache(k8: torch.Tensor, k_scale: torch.Tensor, kv: Optional[torch.Tenso
 
 
 def make_queries(tok_seq: torch.Tensor, tok_pos: torch.Tensor, max_pos: int) -> Queries:
-    q = Queries(tok_seq.shape[0], _ptr(tok_seq), _ptr(tok_pos), int(max_pos))
+    T = tok_seq.shape[0]
+    _check_arg(tok_seq, "tok_seq", DT_I32, (T,))
+    _check_arg(tok_pos, "tok_pos", DT_I32, (T,))
+    q = Queries(T, _ptr(tok_seq), _ptr(tok_pos), int(max_pos))
     q._tensors = (tok_seq, tok_pos)  # the struct holds raw pointers into these
     return q
+
+
+def _check_indexer_args(cache: PagedCache, queries: Queries, q8, q_scale, w, logits):
+    T = queries.n_tokens
+    _check_arg(q8, "q8", DT_FP8, (T, None, cache.idx_dim))
+    _check_arg(q_scale, "q_scale", DT_F32, (T,))
+    _check_arg(w, "w", DT_F32, (T, q8.shape[1]))
+    _check_arg(logits, "logits", DT_F32, (T, None))
+    _check_ld(logits, "logits", queries)
+
+
+def _check_attn_args(cache: PagedCache, queries: Queries, q, d_v: int, k: int, idx, out, lse,
+                     idx_optional: bool = False):
+    T = queries.n_tokens
+    _check_arg(q, "q", DT_BF16, (T, None, cache.d_kv))
+    H = q.shape[1]
+    _check_arg(idx, "idx", DT_I32, (T, k), optional=idx_optional)
+    _check_arg(out, "out", DT_BF16, (T, H, d_v))
+    _check_arg(lse, "lse", DT_F32, (T, H), optional=True)
 
 
 def _workspace(nbytes: int, device) -> torch.Tensor:
@@ -158,6 +219,7 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
 def dsa_indexer_logits(cache: PagedCache, queries: Queries, q8, q_scale, w, logits,
                        workspace=None, stream=None):
     """(1) logits[t, s] = sum_j w[t,j] ReLU(qhat[t,j] . khat[s]) for s <= tok_pos[t]."""
+    _check_indexer_args(cache, queries, q8, q_scale, w, logits)
     T = queries.n_tokens
     need = lib().dsa_indexer_workspace_size(T)
     if workspace is None:
@@ -175,6 +237,7 @@ def dsa_indexer_logits_noalloc(cache: PagedCache, queries: Queries, q8, q_scale,
     """dsa_indexer_logits without a workspace argument, for callers that cannot allocate
     device memory: the library uses its own fixed 256 KiB device array (at most 12288
     query tokens per call; calls that overlap on the GPU share it and race)."""
+    _check_indexer_args(cache, queries, q8, q_scale, w, logits)
     st = lib().dsa_indexer_logits_noalloc(ctypes.byref(cache), ctypes.byref(queries), _ptr(q8),
                                           _ptr(q_scale), _ptr(w), q8.shape[1], _ptr(logits),
                                           logits.shape[1], _stream(stream))
@@ -184,6 +247,9 @@ def dsa_indexer_logits_noalloc(cache: PagedCache, queries: Queries, q8, q_scale,
 
 def dsa_topk(logits, queries: Queries, k: int, idx, workspace=None, stream=None):
     """(2) idx[t, :] = the positions of the k largest logits of row t (-1 padded)."""
+    _check_arg(logits, "logits", DT_F32, (queries.n_tokens, None))
+    _check_ld(logits, "logits", queries)
+    _check_arg(idx, "idx", DT_I32, (queries.n_tokens, k))
     need = lib().dsa_topk_workspace_size(queries.n_tokens, queries.max_pos, k)
     if workspace is None and need:
         workspace = _workspace(need, logits.device)
@@ -197,6 +263,8 @@ def dsa_topk(logits, queries: Queries, k: int, idx, workspace=None, stream=None)
 def dsa_sparse_mla_attn(cache: PagedCache, queries: Queries, q, d_v: int, scale: float, idx,
                         out, lse=None, workspace=None, stream=None):
     """(3) out[t,h] = softmax over the selected latent rows of scale*q.kv, times kv[:, :d_v]."""
+    _check_arg(idx, "idx", DT_I32, (queries.n_tokens, None))
+    _check_attn_args(cache, queries, q, d_v, idx.shape[1], idx, out, lse)
     T, H = q.shape[0], q.shape[1]
     k = idx.shape[1]
     need = lib().dsa_attn_workspace_size(T, H, d_v, k)
@@ -217,6 +285,11 @@ def forward_workspace_size(n_tokens: int, max_pos: int, k: int, n_heads: int, d_
 def dsa_forward(cache: PagedCache, queries: Queries, q8, q_scale, w, q, d_v: int, scale: float,
                 k: int, out, lse=None, idx_out=None, workspace=None, stream=None):
     """(1) + (2) + (3) in one call."""
+    T0 = queries.n_tokens
+    _check_arg(q8, "q8", DT_FP8, (T0, None, cache.idx_dim))
+    _check_arg(q_scale, "q_scale", DT_F32, (T0,))
+    _check_arg(w, "w", DT_F32, (T0, q8.shape[1]))
+    _check_attn_args(cache, queries, q, d_v, k, idx_out, out, lse, idx_optional=True)
     T, H = q.shape[0], q.shape[1]
     need = forward_workspace_size(T, queries.max_pos, k, H, d_v)
     if workspace is None:
@@ -234,6 +307,18 @@ def dsa_cache_append(cache: PagedCache, k8, k_scale, kv, tok_seq, tok_pos, k_in,
     """(0) Write new tokens into the paged caches: k8[r] = e4m3(k_in[i] / s), k_scale[r] = s =
     amax / 448, kv[r] = kv_in[i], r the row of (tok_seq[i], tok_pos[i]) through the block table.
     k_in is fp32 [n_new, idx_dim]; kv_in bf16 bits [n_new, d_kv] or None."""
+    n = tok_seq.shape[0]
+    _check_arg(k8, "k8", DT_FP8, (None, cache.idx_dim))
+    if k8.shape[0] < cache.num_blocks * cache.page_size:
+        raise ValueError(f"k8: {k8.shape[0]} rows < the cache's "
+                         f"{cache.num_blocks * cache.page_size}")
+    _check_arg(k_scale, "k_scale", DT_F32, (k8.shape[0],))
+    _check_arg(tok_seq, "tok_seq", DT_I32, (n,))
+    _check_arg(tok_pos, "tok_pos", DT_I32, (n,))
+    _check_arg(k_in, "k_in", DT_F32, (n, cache.idx_dim))
+    if kv is not None and kv_in is not None:
+        _check_arg(kv, "kv", DT_BF16, (k8.shape[0], cache.d_kv))
+        _check_arg(kv_in, "kv_in", DT_BF16, (n, cache.d_kv))
     st = lib().dsa_cache_append(ctypes.byref(cache), _ptr(k8), _ptr(k_scale), _ptr(kv),
                                 tok_seq.shape[0], _ptr(tok_seq), _ptr(tok_pos), _ptr(k_in),
                                 _ptr(kv_in), _stream(stream))
@@ -244,6 +329,10 @@ def dsa_cp_candidates(logits, idx, pos_offset: int, values, positions, stream=No
     """values[t, j] = logits[t, idx[t, j]], positions[t, j] = idx[t, j] + pos_offset (-inf / -1
     for empty slots)."""
     T, k = idx.shape
+    _check_arg(idx, "idx", DT_I32, (T, k))
+    _check_arg(logits, "logits", DT_F32, (T, None))
+    _check_arg(values, "values", DT_F32, (T, k))
+    _check_arg(positions, "positions", DT_I32, (T, k))
     _check("dsa_cp_candidates",
            lib().dsa_cp_candidates(_ptr(logits), logits.shape[1], T, _ptr(idx), k,
                                    int(pos_offset), _ptr(values), _ptr(positions),
@@ -254,6 +343,10 @@ def dsa_cp_merge_topk(values, positions, k: int, idx_out, local_begin: int = 0,
                       local_end: int = 0, idx_local=None, workspace=None, stream=None):
     """[G, T, k] candidates -> [T, k] global selection (and this part's local view)."""
     G, T, kc = values.shape
+    _check_arg(values, "values", DT_F32, (G, T, k))
+    _check_arg(positions, "positions", DT_I32, (G, T, k))
+    _check_arg(idx_out, "idx_out", DT_I32, (T, k))
+    _check_arg(idx_local, "idx_local", DT_I32, (T, k), optional=True)
     need = int(lib().dsa_cp_merge_workspace_size(T, G, kc))
     if workspace is None:
         workspace = _workspace(need, values.device)
@@ -267,6 +360,10 @@ def dsa_cp_merge_topk(values, positions, k: int, idx_out, local_begin: int = 0,
 def dsa_cp_attn_merge(o_parts, lse_parts, out, lse=None, stream=None):
     """[G, T, H, d_v] bf16 partials + [G, T, H] LSE -> out [T, H, d_v], lse [T, H]."""
     G, T, H, d_v = o_parts.shape
+    _check_arg(o_parts, "o_parts", DT_BF16, (G, T, H, d_v))
+    _check_arg(lse_parts, "lse_parts", DT_F32, (G, T, H))
+    _check_arg(out, "out", DT_BF16, (T, H, d_v))
+    _check_arg(lse, "lse", DT_F32, (T, H), optional=True)
     _check("dsa_cp_attn_merge",
            lib().dsa_cp_attn_merge(_ptr(o_parts), _ptr(lse_parts), G, T, H, d_v, _ptr(out),
                                    _ptr(lse), _stream(stream)))
