@@ -282,9 +282,9 @@ def forward_workspace_size(n_tokens: int, max_pos: int, k: int, n_heads: int, d_
     return int(lib().dsa_forward_workspace_size(n_tokens, max_pos, k, n_heads, d_v))
 
 
-def dsa_forward(cache: PagedCache, queries: Queries, q8, q_scale, w, q, d_v: int, scale: float,
-                k: int, out, lse=None, idx_out=None, workspace=None, stream=None):
-    """(1) + (2) + (3) in one call."""
+def _forward_args(cache: PagedCache, queries: Queries, q8, q_scale, w, q, d_v: int,
+                  scale: float, k: int, out, lse, idx_out, workspace, stream):
+    """Checked, marshalled arguments of dsa_forward, and the workspace they point into."""
     T0 = queries.n_tokens
     _check_arg(q8, "q8", DT_FP8, (T0, None, cache.idx_dim))
     _check_arg(q_scale, "q_scale", DT_F32, (T0,))
@@ -294,12 +294,41 @@ def dsa_forward(cache: PagedCache, queries: Queries, q8, q_scale, w, q, d_v: int
     need = forward_workspace_size(T, queries.max_pos, k, H, d_v)
     if workspace is None:
         workspace = _workspace(need, q.device)
-    st = lib().dsa_forward(ctypes.byref(cache), ctypes.byref(queries), _ptr(q8), _ptr(q_scale),
-                           _ptr(w), q8.shape[1], _ptr(q), H, d_v, float(scale), k, _ptr(out),
-                           _ptr(lse), _ptr(idx_out), _ptr(workspace), workspace.numel(),
-                           _stream(stream))
-    _check("dsa_forward", st)
+    args = (ctypes.byref(cache), ctypes.byref(queries), _ptr(q8), _ptr(q_scale), _ptr(w),
+            q8.shape[1], _ptr(q), H, d_v, float(scale), k, _ptr(out), _ptr(lse), _ptr(idx_out),
+            _ptr(workspace), workspace.numel(), _stream(stream))
+    return args, workspace
+
+
+def dsa_forward(cache: PagedCache, queries: Queries, q8, q_scale, w, q, d_v: int, scale: float,
+                k: int, out, lse=None, idx_out=None, workspace=None, stream=None):
+    """(1) + (2) + (3) in one call."""
+    args, _ = _forward_args(cache, queries, q8, q_scale, w, q, d_v, scale, k, out, lse, idx_out,
+                            workspace, stream)
+    _check("dsa_forward", lib().dsa_forward(*args))
     return out
+
+
+class ForwardCall:
+    """dsa_forward bound once to fixed buffers: the arguments are checked and marshalled
+    here, and each call() is one foreign call.  For a decode loop that rewrites its inputs
+    (q8, q_scale, w, q, the token positions) in place every step, this takes the binding's
+    per-step host cost down to that of the C call itself.  The tensors (and the cache and
+    queries descriptors) must stay allocated and unmoved while the object is used; the
+    object keeps references to them.  Every call runs on the stream given here (default:
+    torch's current stream at construction)."""
+
+    def __init__(self, cache: PagedCache, queries: Queries, q8, q_scale, w, q, d_v: int,
+                 scale: float, k: int, out, lse=None, idx_out=None, workspace=None, stream=None):
+        self._args, ws = _forward_args(cache, queries, q8, q_scale, w, q, d_v, scale, k, out,
+                                       lse, idx_out, workspace, stream)
+        self._keep = (cache, queries, q8, q_scale, w, q, out, lse, idx_out, ws)
+        self._fn = lib().dsa_forward
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != DSA_OK:
+            raise DsaError("dsa_forward", st)
 
 
 def dsa_cache_append(cache: PagedCache, k8, k_scale, kv, tok_seq, tok_pos, k_in, kv_in=None,

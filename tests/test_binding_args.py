@@ -3,7 +3,11 @@ element type and the extents of every tensor) before anything reaches the librar
 wrong tensor raises on the host instead of letting a kernel read or write past its end.
 
 CPU only: the tensors here live on the host, so a call whose arguments all pass the checks
-stops at the next one ("CUDA tensors only") — no device pointer is ever formed."""
+stops at the next one ("CUDA tensors only") — no device pointer is ever formed.  The
+bound-call object (ForwardCall) is checked against dsa_forward with a recording stand-in for
+the library: it must hand the C entry point the same arguments."""
+
+import ctypes
 
 import pytest
 import torch
@@ -156,3 +160,60 @@ def test_context_parallel_arguments():
     _expect("lse_parts: shape", dsa.dsa_cp_attn_merge, o, lp[:, :, :-1], out, lse)
     _expect("out: shape", dsa.dsa_cp_attn_merge, o, lp, out[:-1], lse)
     _expect("o_parts: dtype", dsa.dsa_cp_attn_merge, o.float(), lp, out, lse)
+
+
+class _RecordingLib:
+    """Stands in for libdsa: records each call's arguments and returns DSA_OK."""
+
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        def fn(*args):
+            self.calls.append((name, args))
+            return 1 << 20 if name.endswith("workspace_size") else 0
+        return fn
+
+
+def _norm(a):
+    if hasattr(a, "_obj"):  # ctypes.byref
+        return ("ref", id(a._obj))
+    if isinstance(a, ctypes.c_void_p):
+        return ("ptr", a.value)
+    return a
+
+
+def test_forward_call_marshals_like_dsa_forward(monkeypatch):
+    """ForwardCall passes the C entry point exactly what dsa_forward passes, and each call
+    of the bound object is one call of the entry point."""
+    fake = _RecordingLib()
+    monkeypatch.setattr(dsa, "_LIB", fake)
+    monkeypatch.setattr(dsa, "_ptr", lambda t: None if t is None else ctypes.c_void_p(t.data_ptr()))
+    monkeypatch.setattr(dsa, "_stream", lambda s=None: ctypes.c_void_p(1234))
+    c, q = _cache(), _queries()
+    i, a = _indexer_args(), _attn_args()
+    ws = torch.empty(1 << 20, dtype=torch.uint8)
+    argv = (c, q, i["q8"], i["q_scale"], i["w"], a["q"], DV, 0.07, K, a["out"], a["lse"], a["idx"],
+            ws)
+    dsa.dsa_forward(*argv)
+    direct = [x for x in fake.calls if x[0] == "dsa_forward"]
+    fc = dsa.ForwardCall(*argv)
+    n0 = len(fake.calls)
+    fc()
+    fc()
+    bound = [x for x in fake.calls[n0:] if x[0] == "dsa_forward"]
+    assert len(direct) == 1 and len(bound) == 2 and len(fake.calls) - n0 == 2
+    want = [_norm(x) for x in direct[0][1]]
+    for _, args in bound:
+        assert [_norm(x) for x in args] == want
+    assert len(want) == 17
+
+
+def test_forward_call_checks_its_arguments():
+    c, q = _cache(), _queries()
+    i, a = _indexer_args(), _attn_args()
+    with pytest.raises(ValueError, match="out: shape"):
+        dsa.ForwardCall(c, q, i["q8"], i["q_scale"], i["w"], a["q"], DV, 0.07, K,
+                        torch.zeros(T, H, DV // 2, dtype=torch.int16))
+    with pytest.raises(ValueError, match="CUDA tensors only"):
+        dsa.ForwardCall(c, q, i["q8"], i["q_scale"], i["w"], a["q"], DV, 0.07, K, a["out"])
