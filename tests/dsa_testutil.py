@@ -132,3 +132,32 @@ def oracle_attention(w: DeviceWorkload, t: int, sel: np.ndarray):
     c, q = w.host_cache, w.host_q
     return R.sparse_mla_attn_token(c.kv, c.block_table, int(q.tok_seq[t]), q.q[t], sel,
                                    w.cfg.scale, w.cfg.d_v)
+
+
+# ------------------------------------------------------------------------------ guard regions
+
+GUARD_BYTES = 4096   # a multiple of 256: the interior keeps the allocation's alignment
+GUARD_BYTE = 0xA5
+
+
+class Guarded:
+    """A tensor of `shape` and `dtype` placed inside one larger byte allocation, with
+    GUARD_BYTES of a fixed byte pattern before it and at least that many after it.  A
+    kernel that writes past either end of the tensor changes a guard byte; intact() says
+    whether the guards still hold the pattern.  This stands in for a memory checker."""
+
+    def __init__(self, shape, dtype, device, fill=None):
+        shape = tuple(int(s) for s in shape)
+        elem = torch.empty((), dtype=dtype).element_size()
+        self.nbytes = int(np.prod(shape, dtype=np.int64)) * elem
+        padded = (self.nbytes + 255) // 256 * 256
+        self.buf = torch.full((GUARD_BYTES + padded + GUARD_BYTES,), GUARD_BYTE,
+                              dtype=torch.uint8, device=device)
+        self.t = self.buf[GUARD_BYTES:GUARD_BYTES + self.nbytes].view(dtype).view(shape)
+        if fill is not None:
+            self.t.fill_(fill)
+
+    def intact(self) -> bool:
+        head = self.buf[:GUARD_BYTES]
+        tail = self.buf[GUARD_BYTES + self.nbytes:]
+        return bool((head == GUARD_BYTE).all().item() and (tail == GUARD_BYTE).all().item())
