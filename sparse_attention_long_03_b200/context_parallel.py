@@ -131,14 +131,22 @@ def cp_decode_step(part: Part, st: Step, group=None, ops: Optional[CudaOps] = No
 
 
 def split_parts(block_table: torch.Tensor, k8, k_scale, kv, lengths: List[int], G: int):
-    """Parts of a shared physical cache: part g owns the page-aligned position range
-    [g * P, (g + 1) * P) of every sequence (P = the longest length split G ways, rounded up
-    to whole pages); its block table is the matching column slice of `block_table`."""
-    n_pages = (max(lengths) + PAGE - 1) // PAGE
-    per = (n_pages + G - 1) // G
-    parts = []
-    for g in range(G):
-        c0, c1 = g * per, min((g + 1) * per, block_table.shape[1])
-        bt = block_table[:, c0:c1].contiguous()
-        parts.append(Part(c0 * PAGE, c1 * PAGE, dsa.make_cache(k8, k_scale, kv, bt)))
-    return parts
+    """Parts of a shared physical cache: part g owns a page-aligned position range of every
+    sequence (`part_pages`); its block table is the matching column slice of
+    `block_table`."""
+    return [Part(c0 * PAGE, c1 * PAGE,
+                 dsa.make_cache(k8, k_scale, kv, block_table[:, c0:c1].contiguous()))
+            for c0, c1 in part_pages(max(lengths), block_table.shape[1], G)]
+
+
+def part_pages(max_len: int, table_cols: int, G: int):
+    """Block-table column ranges [c0, c1) of the G parts: the pages holding the longest
+    sequence's positions, split as evenly as whole pages allow.  Every part gets at least
+    one page (a part without keys has nothing to score), so G may not exceed that page
+    count."""
+    n_pages = (max_len + PAGE - 1) // PAGE
+    if G < 1 or n_pages > table_cols:
+        raise ValueError(f"{G} parts of {n_pages} pages with {table_cols} block-table columns")
+    if G > n_pages:
+        raise ValueError(f"{G} parts but only {n_pages} pages: every part needs a page")
+    return [(n_pages * g // G, n_pages * (g + 1) // G) for g in range(G)]

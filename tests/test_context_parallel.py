@@ -130,3 +130,26 @@ def test_two_gloo_ranks_match_the_single_part_oracle():
         for same_sel, o_err, l_err in got[rank]:
             assert same_sel
             assert o_err < 1e-10 and l_err < 1e-10
+
+
+def test_part_pages_cover_the_context_in_order():
+    """The parts' page ranges tile [0, pages) in order, none empty, as even as whole pages
+    allow; more parts than pages, or a context longer than the block table, is an error."""
+    import pytest
+
+    from sparse_attention_long_03_b200.context_parallel import part_pages
+    for max_len, cols in [(32768, 512), (640, 10), (65, 2), (131072, 2048), (100, 5)]:
+        n_pages = (max_len + 63) // 64
+        for G in range(1, n_pages + 1):
+            r = part_pages(max_len, cols, G)
+            assert len(r) == G and r[0][0] == 0 and r[-1][1] == n_pages
+            assert all(a < b for a, b in r)
+            assert all(r[i][1] == r[i + 1][0] for i in range(G - 1))
+            sizes = [b - a for a, b in r]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        part_pages(640, 10, 11)  # more parts than pages
+    with pytest.raises(ValueError):
+        part_pages(640, 9, 2)  # context longer than the block table
+    with pytest.raises(ValueError):
+        part_pages(640, 10, 0)
